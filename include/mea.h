@@ -1,0 +1,146 @@
+/*
+ * mea.h — C ABI of libmea, exact memory-efficient attention for B200 (sm_100a).
+ *
+ * What the library computes (all entry points):
+ *
+ *     out = softmax(Q K^T * scale + bias) V,   lse = log(sum(exp(Q K^T * scale + bias)))
+ *
+ * row by row, over a packed batch of variable-length segments that never attend to one
+ * another (the block-diagonal mask of "Cómo construir transformadores con memoria eficiente
+ * con xFormers…", section 4 "packed variable-length batch", and technique 1 "Packed Sequences &
+ * BlockDiagonalMask" of "How to Build Memory-Efficient Transformers with xFormers…"), optionally
+ * under an implicit lower-triangular causal mask (technique 5 of the latter), with grouped-query
+ * attention (the G key/value heads of "group query attention gqa", each shared by R = Hq/Hkv
+ * query heads; R = Hq is MQA) and an optional per-head ALiBi additive bias (technique 3).
+ * The score matrix is computed tile by tile with an online softmax and never reaches global
+ * memory (the blockwise engine of "大模型推理加速终极指南", section 1).
+ *
+ * Notation and layouts (row-major, contiguous, 16-byte aligned base pointers):
+ *   T_q, T_k   total packed query / key tokens;   Hq, Hkv   query / key-value heads; D head_dim
+ *   q   [T_q, Hq,  D]  fp16 or bf16          out [T_q, Hq, D] same dtype as q
+ *   k,v [T_k, Hkv, D]  same dtype            lse [Hq, T_q] fp32 (natural log), may be NULL
+ *   cu_seqlens_q / cu_seqlens_k: int32 [n_seqs+1] prefix sums of segment lengths, in DEVICE
+ *   memory; segment s owns query rows [cu_q[s], cu_q[s+1]) and key rows [cu_k[s], cu_k[s+1]).
+ *   Query head h reads key/value head h / R (the repeat_interleave grouping).
+ *
+ * Per segment s with L_q = cu_q[s+1]-cu_q[s], L_k = cu_k[s+1]-cu_k[s], query row i sits at key
+ * position p_i = i + L_k - L_q (bottom-right alignment: the last query sees the last key).
+ *   MEA_MASK_NONE:   row i attends to keys j in [0, L_k)
+ *   MEA_MASK_CAUSAL: row i attends to keys j in [0, min(p_i, L_k-1)]
+ *   ALiBi (alibi_slopes != NULL): bias(i, j) = -slope[h] * |p_i - j|, added after scaling.
+ * A row with no admissible key (L_k = 0, or causal with p_i < 0) gets out = 0, lse = -inf.
+ *
+ * Ownership: the caller owns and allocates every buffer; the library never allocates device
+ * memory in these calls. Errors: arguments are validated before anything is launched and a
+ * negative mea_status is returned with nothing launched; MEA_ERR_CUDA reports a failed launch.
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream) and never
+ * synchronise the host.
+ */
+#ifndef MEA_H_
+#define MEA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MEA_OK = 0,
+  MEA_ERR_NULL = -1,          /* a required pointer is NULL                                   */
+  MEA_ERR_SHAPE = -2,         /* negative/zero sizes, total or max_seqlen out of range        */
+  MEA_ERR_HEADS = -3,         /* n_heads_q % n_heads_kv != 0, or a head count < 1             */
+  MEA_ERR_HEAD_DIM = -4,      /* head_dim not in {64, 128}                                    */
+  MEA_ERR_DTYPE = -5,         /* dtype not MEA_F16 / MEA_BF16                                 */
+  MEA_ERR_ALIGN = -6,         /* a tensor base pointer is not 16-byte aligned (TMA needs it)  */
+  MEA_ERR_MASK = -7,          /* mask_kind not a mea_mask value                               */
+  MEA_ERR_WORKSPACE = -8,     /* workspace NULL or smaller than the size function says        */
+  MEA_ERR_CUDA = -9,          /* a CUDA runtime/driver call or a launch failed                */
+  MEA_ERR_DEVICE_TIMEOUT = -10, /* a kernel gave up on a bounded wait (see mea_device_error)  */
+  MEA_ERR_DEVICE = -11,       /* the current device is not an sm_100 part                     */
+  MEA_ERR_SCALE = -12         /* scale is not finite                                           */
+} mea_status;
+
+typedef enum { MEA_F16 = 0, MEA_BF16 = 1 } mea_dtype;
+
+typedef enum {
+  MEA_MASK_NONE = 0,   /* block-diagonal only                                   */
+  MEA_MASK_CAUSAL = 1  /* block-diagonal plus bottom-right lower-triangular    */
+} mea_mask;
+
+/*
+ * mea_forward — packed variable-length attention forward (prefill / training forward).
+ *
+ * Computes out and lse as defined above for every (segment, query row, query head).
+ *   n_seqs        number of segments (>= 1); cu_seqlens_* hold n_seqs+1 entries each.
+ *   total_q/k     T_q = cu_seqlens_q[n_seqs], T_k = cu_seqlens_k[n_seqs] (given by the caller
+ *                 so that the host never reads device memory; they size the TMA views).
+ *   max_seqlen_q  an upper bound on every L_q (sizes the work decomposition; rows past it are
+ *                 not computed, so it must not be smaller than the true maximum).
+ *   scale         multiplies Q K^T before the bias (1/sqrt(D) is the usual choice).
+ *   alibi_slopes  NULL, or DEVICE fp32 [n_heads_q] slopes (2^(-8(h+1)/Hq) is the usual choice).
+ *   dtype         mea_dtype of q, k, v and out.
+ * Returns MEA_OK or a negative mea_status. Segments with L_q = 0 produce nothing.
+ */
+int mea_forward(const void* q, const void* k, const void* v, void* out, float* lse,
+                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int n_seqs,
+                int total_q, int total_k, int max_seqlen_q, int n_heads_q, int n_heads_kv,
+                int head_dim, float scale, int mask_kind, const float* alibi_slopes,
+                int dtype, void* stream);
+
+/*
+ * mea_decode_workspace_size — bytes of device workspace mea_decode_splitkv needs.
+ *   split_keys is the number of keys per split-KV chunk (0 = the library's choice for these
+ *   sizes; pass the same value to mea_decode_splitkv). Returns 0 for invalid arguments.
+ *   The workspace holds, for every chunk, one partial output row and one partial lse per query
+ *   head of the chunk's group, in fp32.
+ */
+size_t mea_decode_workspace_size(int n_seqs, int total_k, int n_heads_q, int n_heads_kv,
+                                 int head_dim, int split_keys);
+
+/*
+ * mea_decode_splitkv — one query token per request against a packed KV cache, split along the
+ * keys (the split-K attention of "大模型推理加速终极指南", section 1) and merged by
+ * log-sum-exp.
+ *   q    [n_seqs, n_heads_q, D]   one token per request      out [n_seqs, n_heads_q, D]
+ *   k,v  [total_k, n_heads_kv, D] packed, request b owns rows [cu_k[b], cu_k[b+1])
+ *   lse  [n_heads_q, n_seqs] fp32 or NULL
+ * The single query is the newest token of its request (p = L_k - 1), so it attends to all L_k
+ * keys; mask_kind is accepted for symmetry and CAUSAL equals NONE here.
+ *   workspace/workspace_bytes: caller-owned device scratch of at least
+ *   mea_decode_workspace_size(...) bytes, 256-byte aligned; its contents need no initialisation.
+ *   split_keys: keys per chunk, a multiple of 64 (0 = library's choice).
+ * Two kernels are launched on `stream`: the split kernel and the log-sum-exp merge kernel.
+ */
+int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, float* lse,
+                       const int32_t* cu_seqlens_k, int n_seqs, int total_k, int max_seqlen_k,
+                       int n_heads_q, int n_heads_kv, int head_dim, float scale, int mask_kind,
+                       const float* alibi_slopes, int dtype, void* workspace,
+                       size_t workspace_bytes, int split_keys, void* stream);
+
+/* mea_status_string — a static English description of a mea_status value. */
+const char* mea_status_string(int status);
+
+/*
+ * mea_device_error — reads (and, if `clear` != 0, resets) the device-side error word of the
+ * current device. Kernels bound every wait; one that gives up records a non-zero code here
+ * (bits 0..7: which wait, bits 8..15: which kernel) and returns early. Synchronises the device.
+ * Returns MEA_OK and stores the word in *code, or MEA_ERR_CUDA.
+ */
+int mea_device_error(int* code, int clear);
+
+/*
+ * mea_set_wait_timeout_ns — the bound, in nanoseconds, on every wait inside the kernels
+ * (default 2e9). Applies to launches made after the call, from any thread.
+ */
+void mea_set_wait_timeout_ns(unsigned long long ns);
+
+/* mea_version — library version string. */
+const char* mea_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEA_H_ */
