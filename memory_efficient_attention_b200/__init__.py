@@ -1,0 +1,247 @@
+"""memory_efficient_attention_b200 — exact memory-efficient attention on B200 (sm_100a).
+
+A thin PyTorch binding over libmea.so (C ABI in include/mea.h). PyTorch supplies device memory
+and the current CUDA stream; every step of the computation runs in the library's kernels. There
+is no CPU path: calling any op without a built library or without an sm_100 GPU raises.
+
+Public API (names follow the pages' vocabulary):
+
+* :func:`memory_efficient_attention` — ``(q, k, v, attn_bias=None, scale=None)`` on BMHK
+  ``[B, M, H, K]`` or BMGHK ``[B, M, G, Hq, K]`` tensors, the call of the 7minutos page's packed
+  and grouped examples; ``attn_bias`` is a :class:`BlockDiagonalMask`,
+  :class:`BlockDiagonalCausalMask` or :class:`LowerTriangularMask`, optionally with ALiBi slopes.
+* :func:`attention_packed` — the raw packed-varlen call ``[T, H, D]`` with ``cu_seqlens``.
+* :func:`decode_splitkv` — one query token per request against a packed KV cache.
+* :func:`alibi_slopes` — ``2^(-8(h+1)/H)``.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import MeaError  # noqa: F401
+
+__all__ = [
+    "memory_efficient_attention", "attention_packed", "decode_splitkv",
+    "decode_workspace_size", "alibi_slopes", "BlockDiagonalMask", "BlockDiagonalCausalMask",
+    "LowerTriangularMask", "device_error", "set_wait_timeout_ns", "MeaError", "library_path",
+]
+
+library_path = _lib.LIB_PATH
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float16:
+        return _lib.MEA_F16
+    if t == torch.bfloat16:
+        return _lib.MEA_BF16
+    raise MeaError(_lib.MEA_ERR_DTYPE, f"dtype {t}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def alibi_slopes(n_heads: int, device=None) -> torch.Tensor:
+    """fp32 ALiBi slopes ``2^(-8(h+1)/H)`` for h = 0..H-1."""
+    return torch.tensor([2.0 ** (-8.0 * (h + 1) / n_heads) for h in range(n_heads)],
+                        dtype=torch.float32, device=device)
+
+
+def _cu(seqlens: Sequence[int], device) -> torch.Tensor:
+    c = [0]
+    for s in seqlens:
+        c.append(c[-1] + int(s))
+    return torch.tensor(c, dtype=torch.int32, device=device)
+
+
+def attention_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                     cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, max_seqlen_q: int,
+                     causal: bool = False, alibi_slopes: Optional[torch.Tensor] = None,
+                     scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, return_lse: bool = True):
+    """Packed varlen attention: q ``[T_q, Hq, D]``, k/v ``[T_k, Hkv, D]``, cu_seqlens int32 on
+    the same device. Returns ``(out [T_q, Hq, D], lse [Hq, T_q] fp32 or None)``."""
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "packed tensors must be [tokens, heads, head_dim]")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise MeaError(_lib.MEA_ERR_DEVICE, "tensors must live on the GPU")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    tq, hq, d = q.shape
+    tk, hkv, _ = k.shape
+    if k.shape != v.shape or k.shape[2] != d or q.dtype != k.dtype or k.dtype != v.dtype:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "q/k/v shapes or dtypes disagree")
+    n_seqs = cu_seqlens_q.numel() - 1
+    if cu_seqlens_k.numel() != n_seqs + 1 or cu_seqlens_q.dtype != torch.int32 \
+            or cu_seqlens_k.dtype != torch.int32:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "cu_seqlens must be int32 [n_seqs+1]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((hq, tq), dtype=torch.float32, device=q.device)
+    if alibi_slopes is not None:
+        alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
+    rc = _lib.load().mea_forward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+        n_seqs, tq, tk, int(max_seqlen_q), hq, hkv, d, float(scale),
+        _lib.MEA_MASK_CAUSAL if causal else _lib.MEA_MASK_NONE, _ptr(alibi_slopes),
+        _dtype_code(q.dtype), _stream(q.device))
+    _lib.check(rc, "mea_forward")
+    return out, lse
+
+
+def decode_workspace_size(n_seqs: int, total_k: int, n_heads_q: int, n_heads_kv: int,
+                          head_dim: int, split_keys: int = 0) -> int:
+    return int(_lib.load().mea_decode_workspace_size(n_seqs, total_k, n_heads_q, n_heads_kv,
+                                                     head_dim, split_keys))
+
+
+def decode_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                   max_seqlen_k: int, alibi_slopes: Optional[torch.Tensor] = None,
+                   scale: Optional[float] = None, split_keys: int = 0,
+                   workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                   lse: Optional[torch.Tensor] = None, return_lse: bool = True):
+    """Single-token decode: q ``[B, Hq, D]`` against packed k/v ``[T_k, Hkv, D]``.
+    Returns ``(out [B, Hq, D], lse [Hq, B] or None)``."""
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "q [B, Hq, D], k/v [T_k, Hkv, D]")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    b, hq, d = q.shape
+    tk, hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ws_bytes = decode_workspace_size(b, tk, hq, hkv, d, split_keys)
+    if ws_bytes == 0:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "mea_decode_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((hq, b), dtype=torch.float32, device=q.device)
+    if alibi_slopes is not None:
+        alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
+    rc = _lib.load().mea_decode_splitkv(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_k), b, tk,
+        int(max_seqlen_k), hq, hkv, d, float(scale), _lib.MEA_MASK_CAUSAL, _ptr(alibi_slopes),
+        _dtype_code(q.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        int(split_keys), _stream(q.device))
+    _lib.check(rc, "mea_decode_splitkv")
+    return out, lse
+
+
+# ------------------------------------------------------------------------------------------
+# Attention-bias descriptors (host objects, like the masks of the 7minutos page, section 4).
+# ------------------------------------------------------------------------------------------
+class BlockDiagonalMask:
+    """Packed segments that never attend to one another. ``q_seqlen[i]`` queries of segment i
+    attend to its ``kv_seqlen[i]`` keys (bottom-right aligned when causal)."""
+    causal = False
+
+    def __init__(self, q_seqlen: Sequence[int], kv_seqlen: Optional[Sequence[int]] = None,
+                 alibi_slopes: Optional[torch.Tensor] = None):
+        self.q_seqlen = [int(x) for x in q_seqlen]
+        self.kv_seqlen = [int(x) for x in (kv_seqlen if kv_seqlen is not None else q_seqlen)]
+        if len(self.kv_seqlen) != len(self.q_seqlen):
+            raise ValueError("q_seqlen and kv_seqlen must have the same length")
+        self.alibi_slopes = alibi_slopes
+        self._dev = {}
+
+    @classmethod
+    def from_seqlens(cls, q_seqlen: Sequence[int], kv_seqlen: Optional[Sequence[int]] = None,
+                     alibi_slopes: Optional[torch.Tensor] = None):
+        return cls(q_seqlen, kv_seqlen, alibi_slopes)
+
+    def cu_seqlens(self, device):
+        key = str(device)
+        if key not in self._dev:
+            self._dev[key] = (_cu(self.q_seqlen, device), _cu(self.kv_seqlen, device))
+        return self._dev[key]
+
+    def split(self, out: torch.Tensor) -> List[torch.Tensor]:
+        """Splits a packed ``[1, T, ...]`` output back into per-segment ``[1, L_i, ...]`` views."""
+        return list(torch.split(out, self.q_seqlen, dim=1))
+
+
+class BlockDiagonalCausalMask(BlockDiagonalMask):
+    """Block-diagonal plus the implicit lower-triangular (bottom-right) mask in each segment."""
+    causal = True
+
+
+class LowerTriangularMask:
+    """Causal mask over each batch row of a BMHK / BMGHK call."""
+    causal = True
+
+    def __init__(self, alibi_slopes: Optional[torch.Tensor] = None):
+        self.alibi_slopes = alibi_slopes
+
+
+def memory_efficient_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                               attn_bias=None, scale: Optional[float] = None) -> torch.Tensor:
+    """Exact attention on BMHK ``[B, M, H, K]`` or BMGHK ``[B, M, G, Hq, K]`` tensors.
+
+    BMGHK: k/v are ``[B, Mk, G, 1, K]`` (one KV head per group, shared by the group's Hq query
+    heads) and the output is ``[B, M, G, Hq, K]``. With a block-diagonal mask B must be 1 and the
+    token axis is the packed concatenation of the mask's segments.
+    """
+    if q.dim() == 5:
+        b, m, g, hq, kd = q.shape
+        if k.dim() != 5 or k.shape[3] != 1 or v.shape != k.shape or k.shape[2] != g:
+            raise MeaError(_lib.MEA_ERR_SHAPE, "BMGHK expects k/v [B, Mk, G, 1, K]")
+        mk = k.shape[1]
+        qp = q.reshape(b * m, g * hq, kd)
+        kp = k.reshape(b * mk, g, kd)
+        vp = v.reshape(b * mk, g, kd)
+        out = _bmhk_packed(qp, kp, vp, b, m, mk, attn_bias, scale)
+        return out.reshape(b, m, g, hq, kd)
+    if q.dim() != 4:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "expected BMHK [B, M, H, K] or BMGHK [B, M, G, Hq, K]")
+    b, m, h, kd = q.shape
+    mk = k.shape[1]
+    out = _bmhk_packed(q.reshape(b * m, h, kd), k.reshape(b * mk, k.shape[2], kd),
+                       v.reshape(b * mk, v.shape[2], kd), b, m, mk, attn_bias, scale)
+    return out.reshape(b, m, h, kd)
+
+
+def _bmhk_packed(qp, kp, vp, b, m, mk, attn_bias, scale):
+    slopes = getattr(attn_bias, "alibi_slopes", None)
+    if isinstance(attn_bias, BlockDiagonalMask):
+        if b != 1:
+            raise MeaError(_lib.MEA_ERR_SHAPE, "block-diagonal masks need B == 1 (packed tokens)")
+        if sum(attn_bias.q_seqlen) != m or sum(attn_bias.kv_seqlen) != mk:
+            raise MeaError(_lib.MEA_ERR_SHAPE, "mask seqlens do not sum to the token count")
+        cu_q, cu_k = attn_bias.cu_seqlens(qp.device)
+        max_q = max(attn_bias.q_seqlen) if attn_bias.q_seqlen else 0
+        causal = attn_bias.causal
+    else:
+        cu_q = torch.arange(0, (b + 1) * m, m, dtype=torch.int32, device=qp.device)
+        cu_k = torch.arange(0, (b + 1) * mk, mk, dtype=torch.int32, device=qp.device)
+        max_q = m
+        causal = isinstance(attn_bias, LowerTriangularMask)
+        if attn_bias is not None and not isinstance(attn_bias, LowerTriangularMask):
+            raise MeaError(_lib.MEA_ERR_MASK, f"unsupported attn_bias {type(attn_bias).__name__}")
+    out, _ = attention_packed(qp, kp, vp, cu_q, cu_k, max_q, causal=causal, alibi_slopes=slopes,
+                              scale=scale, return_lse=False)
+    return out
+
+
+def device_error(clear: bool = True) -> int:
+    """The device-side error word (non-zero if a kernel gave up on a bounded wait)."""
+    import ctypes
+    code = ctypes.c_int(0)
+    _lib.check(_lib.load().mea_device_error(ctypes.byref(code), 1 if clear else 0),
+               "mea_device_error")
+    return code.value
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _lib.load().mea_set_wait_timeout_ns(int(ns))

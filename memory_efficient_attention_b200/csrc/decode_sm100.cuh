@@ -1,0 +1,478 @@
+// decode_sm100.cuh — split-KV single-token decode and its log-sum-exp merge, for sm_100a.
+//
+// The split-K attention of "大模型推理加速终极指南" (section 1): each request's keys are cut into
+// fixed-size chunks; every (chunk, head block) work item produces a chunk-normalised partial
+// output and its log-sum-exp; a second kernel merges the partials of a request by their lse.
+//
+// Split kernel (persistent, 160 threads, one CTA per SM):
+//   warp 4      TMA producer: K and V tiles of 64 keys x D for the item's KV head, NS-slot ring,
+//               streamed continuously across work items.
+//   warps 0-3   consumers: warp w takes keys [16w, 16w+16) of every tile. S = q K^T and
+//               O += P V on mma.sync m16n8k16 (the query rows are the RB <= 16 heads of one KV
+//               group, one token each), online softmax in registers; at the end of an item the
+//               four warps merge their (m, l, O) through shared memory and write the partial.
+// Decode is bound by streaming K/V from HBM (about 8 flop per byte); the small products only need
+// to keep up with that stream, which mma.sync does without loading the FMA pipes.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace mea {
+
+struct DecParams {
+  const void* q;      // [n_seqs, hq, D]
+  void* out;          // [n_seqs, hq, D]
+  float* lse;         // [hq, n_seqs] or null
+  const int32_t* cu_k;
+  const float* slopes;
+  float* ws_o;        // [n_slots, hq, D]
+  float* ws_lse;      // [n_slots, hq]
+  int n_seqs;
+  int hq;
+  int R;              // query heads per KV head
+  int RB;             // query heads per work item (<= 16, divides R)
+  int n_hb;           // hq / RB
+  int chunk;          // keys per chunk, a multiple of 64
+  int n_slots;        // upper bound on the number of chunks
+  long long n_items;  // n_slots * n_hb
+  float c1;           // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct DecCfg {
+  static constexpr int BK = 64;                       // keys per tile
+  static constexpr int ATOMS = D / 64;
+  static constexpr uint32_t ATOM_BYTES = BK * 128;    // 64 keys x 128 B
+  static constexpr uint32_t KT_BYTES = BK * D * 2;    // one K (or V) tile
+  static constexpr uint32_t STAGE_BYTES = 2 * KT_BYTES;
+  static constexpr int NS = (D == 128) ? 5 : 8;
+  static constexpr uint32_t SMEM_RING = 0;
+  static constexpr uint32_t SMEM_MERGE = NS * STAGE_BYTES;            // 4 warps x 16 rows x D
+  static constexpr uint32_t MERGE_O_BYTES = 4 * 16 * D * 4;
+  static constexpr uint32_t SMEM_ML = SMEM_MERGE + MERGE_O_BYTES;     // 4 warps x 16 x (m, l)
+  static constexpr uint32_t SMEM_BAR = SMEM_ML + 4 * 16 * 2 * 4;
+  static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
+  static constexpr int THREADS = 160;
+};
+
+// Number of chunks of request i.
+__device__ __forceinline__ int dec_nchunks(const int32_t* cu, int i, int chunk) {
+  const int L = __ldg(cu + i + 1) - __ldg(cu + i);
+  return (L + chunk - 1) / chunk;
+}
+
+// Warp-cooperative: maps a flat chunk id to (request b, chunk c of b); b = -1 past the end.
+__device__ __forceinline__ void dec_find_chunk(const int32_t* cu, int n, int chunk, int cid,
+                                               int& b, int& c) {
+  const int lane = threadIdx.x & 31;
+  int base = 0;
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int i = i0 + lane;
+    const int cnt = i < n ? dec_nchunks(cu, i, chunk) : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int excl = incl - cnt;
+    const bool hit = (i < n) && cid >= base + excl && cid < base + incl;
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (m) {
+      const int src = __ffs(m) - 1;
+      b = i0 + src;
+      c = cid - base - __shfl_sync(0xffffffffu, excl, src);
+      return;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  b = -1;
+  c = 0;
+}
+
+// Warp-cooperative: first flat chunk id of request b.
+__device__ __forceinline__ int dec_chunk_start(const int32_t* cu, int b, int chunk) {
+  const int lane = threadIdx.x & 31;
+  int acc = 0;
+  for (int i0 = 0; i0 < b; i0 += 32) {
+    const int i = i0 + lane;
+    acc += (i < b) ? dec_nchunks(cu, i, chunk) : 0;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  return acc;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+template <bool BF16>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  if constexpr (BF16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t dpack2(float lo, float hi) {
+  if constexpr (BF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+template <int D, bool BF16, bool ALIBI>
+__global__ void __launch_bounds__(160, 1)
+    mea_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
+  using C = DecCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = smem_u32(smem);
+  float* merge_o = reinterpret_cast<float*>(smem + C::SMEM_MERGE);
+  float* merge_ml = reinterpret_cast<float*>(smem + C::SMEM_ML);
+  const uint32_t bar0 = sbase + C::SMEM_BAR;
+#define DBAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+  // B_M0 / B_M1: the four consumer warps' rendezvous before / after the partial merge.
+  constexpr int B_F = 0, B_E = C::NS, B_M0 = 2 * C::NS, B_M1 = B_M0 + 1, N_BARS = B_M1 + 1;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_BAR + 8 * N_BARS);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t tmo = p.timeout_ns;
+  const unsigned ecode = KID_DECODE << 8;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(DBAR(B_F + s), 1);
+      mbar_init(DBAR(B_E + s), 4);
+    }
+    mbar_init(DBAR(B_M0), 128);
+    mbar_init(DBAR(B_M1), 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    uint32_t cnt = 0;
+    bool ok = true;
+    for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
+      const int cid = static_cast<int>(lin / p.n_hb);
+      const int hb = static_cast<int>(lin - static_cast<long long>(cid) * p.n_hb);
+      int b, c;
+      dec_find_chunk(p.cu_k, p.n_seqs, p.chunk, cid, b, c);
+      if (b < 0) break;  // flat chunk ids only grow along this CTA's sequence
+      const int k0 = __ldg(p.cu_k + b);
+      const int L = __ldg(p.cu_k + b + 1) - k0;
+      const int key0 = c * p.chunk;
+      const int nk = min(p.chunk, L - key0);
+      const int n_tiles = (nk + C::BK - 1) / C::BK;
+      const int g = (hb * p.RB) / p.R;
+      if (lane == 0) {
+        for (int t = 0; t < n_tiles; ++t) {
+          const uint32_t s = cnt % C::NS;
+          const uint32_t ph = (cnt / C::NS) & 1u;
+          ok = mbar_wait(DBAR(B_E + s), ph ^ 1u, abort_flag, tmo, ecode | 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(DBAR(B_F + s), C::STAGE_BYTES);
+          const uint32_t dst = sbase + C::SMEM_RING + s * C::STAGE_BYTES;
+          const int tok = k0 + key0 + t * C::BK;
+#pragma unroll
+          for (int a = 0; a < C::ATOMS; ++a) {
+            tma_load_3d(dst + a * C::ATOM_BYTES, &tm_k, DBAR(B_F + s), a * 64, g, tok);
+            tma_load_3d(dst + C::KT_BYTES + a * C::ATOM_BYTES, &tm_v, DBAR(B_F + s), a * 64, g,
+                        tok);
+          }
+          ++cnt;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      cnt = __shfl_sync(0xffffffffu, cnt, 0);
+    }
+    if (!ok && lane == 0) {
+      for (uint32_t s = 0; s < C::NS && s < cnt; ++s) {
+        const uint32_t last = cnt - 1 - ((cnt - 1 - s) % C::NS);
+        volatile int never = 0;
+        mbar_wait(DBAR(B_F + s), (last / C::NS) & 1u, &never, tmo, ecode | 15);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ consumers (warps 0-3)
+    constexpr float LOG2E = 1.4426950408889634f;
+    constexpr float LN2 = 0.6931471805599453f;
+    const int g8 = lane >> 2;  // fragment row (head) 0..7
+    const int t4 = lane & 3;   // fragment column pair
+    uint32_t cnt = 0, n_done = 0;
+    bool ok = true;
+    for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
+      const int cid = static_cast<int>(lin / p.n_hb);
+      const int hb = static_cast<int>(lin - static_cast<long long>(cid) * p.n_hb);
+      int b, c;
+      dec_find_chunk(p.cu_k, p.n_seqs, p.chunk, cid, b, c);
+      if (b < 0) break;
+      const int L = __ldg(p.cu_k + b + 1) - __ldg(p.cu_k + b);
+      const int key0 = c * p.chunk;
+      const int nk = min(p.chunk, L - key0);
+      const int n_tiles = (nk + C::BK - 1) / C::BK;
+      const int pos = L - 1;  // the query is the newest token of its request
+      // q fragments: rows g8 and g8+8 are heads hb*RB + row (zero when row >= RB).
+      const int h_lo = hb * p.RB + g8, h_hi = hb * p.RB + g8 + 8;
+      const bool v_lo = g8 < p.RB, v_hi = g8 + 8 < p.RB;
+      uint32_t qa[D / 16][4];
+      {
+        const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
+        const size_t rlo = (static_cast<size_t>(b) * p.hq + h_lo) * (D / 2);
+        const size_t rhi = (static_cast<size_t>(b) * p.hq + h_hi) * (D / 2);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          qa[kk][0] = v_lo ? __ldg(q32 + rlo + kk * 8 + t4) : 0u;
+          qa[kk][1] = v_hi ? __ldg(q32 + rhi + kk * 8 + t4) : 0u;
+          qa[kk][2] = v_lo ? __ldg(q32 + rlo + kk * 8 + 4 + t4) : 0u;
+          qa[kk][3] = v_hi ? __ldg(q32 + rhi + kk * 8 + 4 + t4) : 0u;
+        }
+      }
+      float sl_lo = 0.f, sl_hi = 0.f;
+      if constexpr (ALIBI) {
+        sl_lo = v_lo ? __ldg(p.slopes + h_lo) * LOG2E : 0.f;
+        sl_hi = v_hi ? __ldg(p.slopes + h_hi) * LOG2E : 0.f;
+      }
+      float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+      float o[D / 8][4];
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+
+      for (int t = 0; t < n_tiles; ++t) {
+        const uint32_t s = cnt % C::NS;
+        const uint32_t ph = (cnt / C::NS) & 1u;
+        ok = mbar_wait(DBAR(B_F + s), ph, abort_flag, tmo, ecode | 2);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const uint32_t kst = sbase + C::SMEM_RING + s * C::STAGE_BYTES;
+        const uint32_t vst = kst + C::KT_BYTES;
+        // ---- S^T fragment: rows = heads, cols = this warp's 16 keys (two n-tiles of 8)
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+          const int kr = warp * 16 + ((lane >> 4) << 3) + (lane & 7);  // key row in the tile
+          const int csel = (lane >> 3) & 1;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int ch = 2 * kk + csel;  // 16-byte chunk along D
+            const uint32_t addr = kst + (ch >> 3) * C::ATOM_BYTES + kr * 128 +
+                                  ((((ch & 7) ^ (kr & 7))) << 4);
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4(addr, r0, r1, r2, r3);
+            mma16816<BF16>(sc[0], qa[kk], r0, r1);
+            mma16816<BF16>(sc[1], qa[kk], r2, r3);
+          }
+        }
+        // ---- online softmax over the 16 keys (rows g8 / g8+8)
+        const int kbase = key0 + t * C::BK + warp * 16;  // key index (in request) of col 0
+        float x[2][4];
+        float mx_lo = -INFINITY, mx_hi = -INFINITY;
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = kbase + n * 8 + 2 * t4 + e;
+            const bool kv = key < key0 + nk;
+            float a = sc[n][e] * p.c1, bb = sc[n][2 + e] * p.c1;
+            if constexpr (ALIBI) {
+              const float dist = static_cast<float>(pos - key);
+              a = fmaf(-sl_lo, dist, a);
+              bb = fmaf(-sl_hi, dist, bb);
+            }
+            x[n][e] = kv ? a : -INFINITY;
+            x[n][2 + e] = kv ? bb : -INFINITY;
+            mx_lo = fmaxf(mx_lo, x[n][e]);
+            mx_hi = fmaxf(mx_hi, x[n][2 + e]);
+          }
+        }
+#pragma unroll
+        for (int off = 1; off <= 2; off <<= 1) {
+          mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, off));
+          mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, off));
+        }
+        const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
+        const float al_lo = (mn_lo == -INFINITY) ? 1.f : ex2_approx(m_lo - mn_lo);
+        const float al_hi = (mn_hi == -INFINITY) ? 1.f : ex2_approx(m_hi - mn_hi);
+        const float mu_lo = (mn_lo == -INFINITY) ? 0.f : mn_lo;
+        const float mu_hi = (mn_hi == -INFINITY) ? 0.f : mn_hi;
+        m_lo = mn_lo;
+        m_hi = mn_hi;
+        float pr[2][4];
+        float s_lo = 0.f, s_hi = 0.f;
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            pr[n][e] = ex2_approx(x[n][e] - mu_lo);
+            pr[n][2 + e] = ex2_approx(x[n][2 + e] - mu_hi);
+            s_lo += pr[n][e];
+            s_hi += pr[n][2 + e];
+          }
+        }
+        l_lo = l_lo * al_lo + s_lo;
+        l_hi = l_hi * al_hi + s_hi;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][0] *= al_lo;
+          o[n][1] *= al_lo;
+          o[n][2] *= al_hi;
+          o[n][3] *= al_hi;
+        }
+        uint32_t pa[4];
+        pa[0] = dpack2<BF16>(pr[0][0], pr[0][1]);
+        pa[1] = dpack2<BF16>(pr[0][2], pr[0][3]);
+        pa[2] = dpack2<BF16>(pr[1][0], pr[1][1]);
+        pa[3] = dpack2<BF16>(pr[1][2], pr[1][3]);
+        // ---- O += P V over this warp's 16 keys
+        {
+          const int kr = warp * 16 + (((lane >> 3) & 1) << 3) + (lane & 7);
+          const int csel = lane >> 4;
+#pragma unroll
+          for (int n = 0; n < D / 8; n += 2) {
+            const int ch = n + csel;
+            const uint32_t addr = vst + (ch >> 3) * C::ATOM_BYTES + kr * 128 +
+                                  ((((ch & 7) ^ (kr & 7))) << 4);
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_t(addr, r0, r1, r2, r3);
+            mma16816<BF16>(o[n], pa, r0, r1);
+            mma16816<BF16>(o[n + 1], pa, r2, r3);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(DBAR(B_E + s));
+        ++cnt;
+      }
+      if (!ok) break;
+      // ---- merge the four warps' partial states and write this item's partial
+      l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+      l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+      float* mo = merge_o + warp * 16 * D;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        mo[g8 * D + n * 8 + 2 * t4] = o[n][0];
+        mo[g8 * D + n * 8 + 2 * t4 + 1] = o[n][1];
+        mo[(g8 + 8) * D + n * 8 + 2 * t4] = o[n][2];
+        mo[(g8 + 8) * D + n * 8 + 2 * t4 + 1] = o[n][3];
+      }
+      if (t4 == 0) {
+        merge_ml[(warp * 16 + g8) * 2 + 0] = m_lo;
+        merge_ml[(warp * 16 + g8) * 2 + 1] = l_lo;
+        merge_ml[(warp * 16 + g8 + 8) * 2 + 0] = m_hi;
+        merge_ml[(warp * 16 + g8 + 8) * 2 + 1] = l_hi;
+      }
+      mbar_arrive(DBAR(B_M0));
+      ok = mbar_wait(DBAR(B_M0), n_done & 1u, abort_flag, tmo, ecode | 3);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      for (int idx = threadIdx.x; idx < p.RB * D; idx += 128) {
+        const int row = idx / D, d = idx - row * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, merge_ml[(w * 16 + row) * 2]);
+        float Lsum = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float wt = ex2_approx(merge_ml[(w * 16 + row) * 2] - M);
+            Lsum += merge_ml[(w * 16 + row) * 2 + 1] * wt;
+            acc += merge_o[(w * 16 + row) * D + d] * wt;
+          }
+        }
+        const int head = hb * p.RB + row;
+        const size_t slot = static_cast<size_t>(cid) * p.hq + head;
+        p.ws_o[slot * D + d] = Lsum > 0.f ? acc / Lsum : 0.f;
+        if (d == 0) p.ws_lse[slot] = Lsum > 0.f ? (M + __log2f(Lsum)) * LN2 : -INFINITY;
+      }
+      mbar_arrive(DBAR(B_M1));
+      ok = mbar_wait(DBAR(B_M1), n_done & 1u, abort_flag, tmo, ecode | 4);
+      ok = __all_sync(0xffffffffu, ok);
+      ++n_done;
+    }
+  }
+#undef DBAR
+  __syncthreads();
+}
+
+// Merge kernel: one CTA per (request, KV group); lse = ln sum_c exp(lse_c),
+// out = sum_c exp(lse_c - lse) O_c, cast to the output dtype.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128)
+    mea_lse_merge_kernel(const DecParams p) {
+  const int b = blockIdx.x;
+  const int g = blockIdx.y;
+  __shared__ int s_start;
+  const int L = __ldg(p.cu_k + b + 1) - __ldg(p.cu_k + b);
+  const int n = (L + p.chunk - 1) / p.chunk;
+  if (threadIdx.x < 32) {
+    const int st = dec_chunk_start(p.cu_k, b, p.chunk);
+    if (threadIdx.x == 0) s_start = st;
+  }
+  __syncthreads();
+  const int c0 = s_start;
+  using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  OutT* out = reinterpret_cast<OutT*>(p.out);
+  for (int idx = threadIdx.x; idx < p.R * D; idx += blockDim.x) {
+    const int r = idx / D, d = idx - r * D;
+    const int head = g * p.R + r;
+    float M = -INFINITY;
+    for (int c = 0; c < n; ++c)
+      M = fmaxf(M, p.ws_lse[static_cast<size_t>(c0 + c) * p.hq + head]);
+    float z = 0.f, acc = 0.f;
+    if (M != -INFINITY) {
+      for (int c = 0; c < n; ++c) {
+        const size_t slot = static_cast<size_t>(c0 + c) * p.hq + head;
+        const float w = __expf(p.ws_lse[slot] - M);
+        z += w;
+        acc += w * p.ws_o[slot * D + d];
+      }
+    }
+    const float val = z > 0.f ? acc / z : 0.f;
+    if constexpr (BF16)
+      out[(static_cast<size_t>(b) * p.hq + head) * D + d] = __float2bfloat16_rn(val);
+    else
+      out[(static_cast<size_t>(b) * p.hq + head) * D + d] = __float2half_rn(val);
+    if (d == 0 && p.lse)
+      p.lse[static_cast<size_t>(head) * p.n_seqs + b] = z > 0.f ? M + __logf(z) : -INFINITY;
+  }
+}
+
+}  // namespace mea

@@ -1,0 +1,360 @@
+// mea_api.cu — the C ABI of libmea (declared in include/mea.h): argument validation, TMA
+// descriptor encoding and kernel launches. No device memory is allocated here; no call
+// synchronises the host except mea_device_error.
+#include <cudaTypedefs.h>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/mea.h"
+#include "decode_sm100.cuh"
+#include "fwd_sm100.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+
+struct DeviceInfo {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device_info(DeviceInfo& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MEA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MEA_ERR_CUDA;
+    d.ok = (major == 10);
+    d.sms = sms;
+    d.init = true;
+  }
+  out = d;
+  return d.ok ? MEA_OK : MEA_ERR_DEVICE;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }();
+  return fn;
+}
+
+// 3-D tiled map over a row-major [d2, d1, d0] tensor of 16-bit elements, 128-byte swizzle.
+bool encode_3d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, dtype == MEA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int largest_pow2_divisor(int x, int cap) {
+  int p = 1;
+  while (p * 2 <= cap && x % (p * 2) == 0) p *= 2;
+  return p;
+}
+
+// ------------------------------------------------------------------------------------------
+// Forward launch dispatch.
+// ------------------------------------------------------------------------------------------
+template <int D, bool BF16, bool CAUSAL, bool ALIBI>
+int launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const mea::FwdParams& p, int grid, cudaStream_t stream) {
+  auto kern = mea::mea_fwd_sm100_kernel<D, BF16, CAUSAL, ALIBI>;
+  constexpr uint32_t smem = mea::FwdCfg<D>::SMEM_TOTAL;
+  static std::once_flag once[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(once[dev], [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return MEA_ERR_CUDA;
+  kern<<<grid, mea::FwdCfg<D>::THREADS, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+int launch_fwd_d(bool causal, bool alibi, const CUtensorMap& tq, const CUtensorMap& tk,
+                 const CUtensorMap& tv, const mea::FwdParams& p, int grid, cudaStream_t s) {
+  if (causal)
+    return alibi ? launch_fwd_t<D, BF16, true, true>(tq, tk, tv, p, grid, s)
+                 : launch_fwd_t<D, BF16, true, false>(tq, tk, tv, p, grid, s);
+  return alibi ? launch_fwd_t<D, BF16, false, true>(tq, tk, tv, p, grid, s)
+               : launch_fwd_t<D, BF16, false, false>(tq, tk, tv, p, grid, s);
+}
+
+// ------------------------------------------------------------------------------------------
+// Decode launch dispatch.
+// ------------------------------------------------------------------------------------------
+template <int D, bool BF16, bool ALIBI>
+int launch_dec_t(const CUtensorMap& tk, const CUtensorMap& tv, const mea::DecParams& p,
+                 int grid, int n_kv_heads, cudaStream_t stream) {
+  auto kern = mea::mea_decode_split_kernel<D, BF16, ALIBI>;
+  constexpr uint32_t smem = mea::DecCfg<D>::SMEM_TOTAL;
+  static std::once_flag once[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(once[dev], [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return MEA_ERR_CUDA;
+  if (grid > 0) kern<<<grid, mea::DecCfg<D>::THREADS, smem, stream>>>(tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return MEA_ERR_CUDA;
+  dim3 mgrid(p.n_seqs, n_kv_heads);
+  mea::mea_lse_merge_kernel<D, BF16><<<mgrid, 128, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+int launch_dec_d(bool alibi, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const mea::DecParams& p, int grid, int hkv, cudaStream_t s) {
+  return alibi ? launch_dec_t<D, BF16, true>(tk, tv, p, grid, hkv, s)
+               : launch_dec_t<D, BF16, false>(tk, tv, p, grid, hkv, s);
+}
+
+int auto_split_keys(int total_k, int n_hb, int sms) {
+  long long work = static_cast<long long>(total_k) * n_hb;
+  long long target = work / (static_cast<long long>(sms > 0 ? sms : 148) * 32);
+  int c = 128;
+  while (c < 2048 && c * 2 <= target) c *= 2;
+  return c;
+}
+
+int decode_rb(int R) {
+  int rb = 1;
+  for (int d = 1; d <= 16; ++d)
+    if (R % d == 0) rb = d;
+  return rb;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct DecLayout {
+  int chunk = 0, n_slots = 0;
+  size_t o_bytes = 0, lse_off = 0, total = 0;
+};
+
+bool dec_layout(int n_seqs, int total_k, int hq, int hkv, int d, int split_keys, int sms,
+                DecLayout& L) {
+  if (n_seqs < 1 || total_k < 0 || hq < 1 || hkv < 1 || hq % hkv || (d != 64 && d != 128))
+    return false;
+  if (split_keys < 0 || split_keys % 64) return false;
+  const int R = hq / hkv;
+  const int n_hb = hq / decode_rb(R);
+  L.chunk = split_keys ? split_keys : auto_split_keys(total_k, n_hb, sms);
+  const long long slots = (static_cast<long long>(total_k) + L.chunk - 1) / L.chunk + n_seqs;
+  if (slots > (1ll << 30)) return false;
+  L.n_slots = static_cast<int>(slots);
+  L.o_bytes = static_cast<size_t>(slots) * hq * d * sizeof(float);
+  L.lse_off = align_up(L.o_bytes, 256);
+  L.total = L.lse_off + align_up(static_cast<size_t>(slots) * hq * sizeof(float), 256);
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mea_version(void) { return "mea 0.1.0 (sm_100a)"; }
+
+const char* mea_status_string(int status) {
+  switch (status) {
+    case MEA_OK: return "MEA_OK: success";
+    case MEA_ERR_NULL: return "MEA_ERR_NULL: a required pointer is NULL";
+    case MEA_ERR_SHAPE: return "MEA_ERR_SHAPE: invalid sizes";
+    case MEA_ERR_HEADS: return "MEA_ERR_HEADS: n_heads_q must be a positive multiple of n_heads_kv";
+    case MEA_ERR_HEAD_DIM: return "MEA_ERR_HEAD_DIM: head_dim must be 64 or 128";
+    case MEA_ERR_DTYPE: return "MEA_ERR_DTYPE: dtype must be MEA_F16 or MEA_BF16";
+    case MEA_ERR_ALIGN: return "MEA_ERR_ALIGN: tensor base pointers must be 16-byte aligned";
+    case MEA_ERR_MASK: return "MEA_ERR_MASK: mask_kind is not a mea_mask value";
+    case MEA_ERR_WORKSPACE: return "MEA_ERR_WORKSPACE: workspace missing or too small";
+    case MEA_ERR_CUDA: return "MEA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case MEA_ERR_DEVICE_TIMEOUT: return "MEA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+    case MEA_ERR_DEVICE: return "MEA_ERR_DEVICE: the current device is not sm_100";
+    case MEA_ERR_SCALE: return "MEA_ERR_SCALE: scale must be finite";
+    default: return "unknown mea_status";
+  }
+}
+
+void mea_set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns.store(ns ? ns : 1ull); }
+
+int mea_device_error(int* code, int clear) {
+  if (!code) return MEA_ERR_NULL;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MEA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, mea::g_mea_error, sizeof(v)) != cudaSuccess) return MEA_ERR_CUDA;
+  *code = static_cast<int>(v);
+  if (clear) {
+    unsigned int z = 0;
+    if (cudaMemcpyToSymbol(mea::g_mea_error, &z, sizeof(z)) != cudaSuccess) return MEA_ERR_CUDA;
+  }
+  return MEA_OK;
+}
+
+int mea_forward(const void* q, const void* k, const void* v, void* out, float* lse,
+                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int n_seqs,
+                int total_q, int total_k, int max_seqlen_q, int n_heads_q, int n_heads_kv,
+                int head_dim, float scale, int mask_kind, const float* alibi_slopes, int dtype,
+                void* stream) {
+  if (!q || !k || !v || !out || !cu_seqlens_q || !cu_seqlens_k) return MEA_ERR_NULL;
+  if (n_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_q > total_q)
+    return MEA_ERR_SHAPE;
+  if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
+  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
+  if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
+  if (!std::isfinite(scale)) return MEA_ERR_SCALE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
+      (alibi_slopes && !aligned(alibi_slopes, 4)))
+    return MEA_ERR_ALIGN;
+  DeviceInfo di;
+  if (int rc = current_device_info(di); rc != MEA_OK) return rc;
+  if (total_q == 0 || max_seqlen_q == 0) return MEA_OK;
+
+  const int R = n_heads_q / n_heads_kv;
+  const int P = largest_pow2_divisor(R, 128);
+  mea::FwdParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.slopes = alibi_slopes;
+  p.n_seqs = n_seqs;
+  p.total_q = total_q;
+  p.hq = n_heads_q;
+  p.P = P;
+  p.R = R;
+  p.n_hb = n_heads_q / P;
+  p.tok_per_tile = 128 / P;
+  p.t_max = (max_seqlen_q + p.tok_per_tile - 1) / p.tok_per_tile;
+  p.n_items = static_cast<long long>(p.t_max) * n_seqs * p.n_hb;
+  p.c1 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t tk_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
+  if (!encode_3d(&tq, q, dtype, head_dim, n_heads_q, total_q, 64, P, 128 / P) ||
+      !encode_3d(&tk, k, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 128) ||
+      !encode_3d(&tv, v, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 128))
+    return MEA_ERR_CUDA;
+  const int grid = static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool causal = mask_kind == MEA_MASK_CAUSAL;
+  const bool alibi = alibi_slopes != nullptr;
+  if (head_dim == 128)
+    return dtype == MEA_BF16 ? launch_fwd_d<128, true>(causal, alibi, tq, tk, tv, p, grid, s)
+                             : launch_fwd_d<128, false>(causal, alibi, tq, tk, tv, p, grid, s);
+  return dtype == MEA_BF16 ? launch_fwd_d<64, true>(causal, alibi, tq, tk, tv, p, grid, s)
+                           : launch_fwd_d<64, false>(causal, alibi, tq, tk, tv, p, grid, s);
+}
+
+size_t mea_decode_workspace_size(int n_seqs, int total_k, int n_heads_q, int n_heads_kv,
+                                 int head_dim, int split_keys) {
+  DeviceInfo di;
+  int sms = (current_device_info(di) == MEA_OK) ? di.sms : 148;
+  DecLayout L;
+  if (!dec_layout(n_seqs, total_k, n_heads_q, n_heads_kv, head_dim, split_keys, sms, L)) return 0;
+  return L.total;
+}
+
+int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, float* lse,
+                       const int32_t* cu_seqlens_k, int n_seqs, int total_k, int max_seqlen_k,
+                       int n_heads_q, int n_heads_kv, int head_dim, float scale, int mask_kind,
+                       const float* alibi_slopes, int dtype, void* workspace,
+                       size_t workspace_bytes, int split_keys, void* stream) {
+  if (!q || !k || !v || !out || !cu_seqlens_k) return MEA_ERR_NULL;
+  if (n_seqs < 1 || total_k < 0 || max_seqlen_k < 0 || max_seqlen_k > total_k)
+    return MEA_ERR_SHAPE;
+  if (split_keys < 0 || split_keys % 64) return MEA_ERR_SHAPE;
+  if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
+  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
+  if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
+  if (!std::isfinite(scale)) return MEA_ERR_SCALE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)) || !aligned(cu_seqlens_k, 4) ||
+      (alibi_slopes && !aligned(alibi_slopes, 4)))
+    return MEA_ERR_ALIGN;
+  if (!workspace || !aligned(workspace, 256)) return MEA_ERR_WORKSPACE;
+  // The automatic chunk size depends on the SM count; an explicit one does not, so a
+  // too-small workspace is reported before the device is queried.
+  DeviceInfo di;
+  int dev_rc = MEA_OK;
+  if (split_keys == 0 && (dev_rc = current_device_info(di)) != MEA_OK) return dev_rc;
+  DecLayout L;
+  if (!dec_layout(n_seqs, total_k, n_heads_q, n_heads_kv, head_dim, split_keys,
+                  split_keys == 0 ? di.sms : 0, L))
+    return MEA_ERR_SHAPE;
+  if (workspace_bytes < L.total) return MEA_ERR_WORKSPACE;
+  if (split_keys != 0 && (dev_rc = current_device_info(di)) != MEA_OK) return dev_rc;
+
+  const int R = n_heads_q / n_heads_kv;
+  mea::DecParams p{};
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.cu_k = cu_seqlens_k;
+  p.slopes = alibi_slopes;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.lse_off);
+  p.n_seqs = n_seqs;
+  p.hq = n_heads_q;
+  p.R = R;
+  p.RB = decode_rb(R);
+  p.n_hb = n_heads_q / p.RB;
+  p.chunk = L.chunk;
+  p.n_slots = L.n_slots;
+  p.n_items = static_cast<long long>(L.n_slots) * p.n_hb;
+  p.c1 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+
+  CUtensorMap tk, tv;
+  const uint64_t tk_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
+  if (!encode_3d(&tk, k, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 64) ||
+      !encode_3d(&tv, v, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 64))
+    return MEA_ERR_CUDA;
+  const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool alibi = alibi_slopes != nullptr;
+  if (head_dim == 128)
+    return dtype == MEA_BF16 ? launch_dec_d<128, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+                             : launch_dec_d<128, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
+  return dtype == MEA_BF16 ? launch_dec_d<64, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+                           : launch_dec_d<64, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,136 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point include/mea.h
+declares, and rejects bad arguments with the documented status before launching anything.
+No GPU is needed: every call here fails argument validation before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from memory_efficient_attention_b200 import _lib
+from memory_efficient_attention_b200.build import build_library
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_library()
+    return _lib.load()
+
+
+def declared_entry_points():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(mea_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = declared_entry_points()
+    assert "mea_forward" in declared and "mea_decode_splitkv" in declared
+    for name in declared:
+        assert hasattr(lib, name), f"libmea.so does not export {name}"
+    assert set(_lib.EXPORTS) <= set(declared)
+
+
+def test_status_strings(lib):
+    for rc in range(0, -13, -1):
+        s = _lib.status_string(rc)
+        assert s and "unknown" not in s
+    assert "unknown" in _lib.status_string(-999)
+    assert lib.mea_version().decode().startswith("mea")
+
+
+A = 0x10000  # an aligned dummy address: never dereferenced, validation fails first
+
+
+def fwd(lib, **kw):
+    args = dict(q=A, k=A, v=A, out=A, lse=A, cu_q=A, cu_k=A, n_seqs=1, total_q=8, total_k=8,
+                max_q=8, hq=8, hkv=2, d=64, scale=0.125, mask=0, slopes=None, dtype=1, stream=None)
+    args.update(kw)
+    return lib.mea_forward(args["q"], args["k"], args["v"], args["out"], args["lse"],
+                           args["cu_q"], args["cu_k"], args["n_seqs"], args["total_q"],
+                           args["total_k"], args["max_q"], args["hq"], args["hkv"], args["d"],
+                           args["scale"], args["mask"], args["slopes"], args["dtype"],
+                           args["stream"])
+
+
+@pytest.mark.parametrize("kw,rc", [
+    (dict(q=None), _lib.MEA_ERR_NULL),
+    (dict(cu_k=None), _lib.MEA_ERR_NULL),
+    (dict(n_seqs=0), _lib.MEA_ERR_SHAPE),
+    (dict(total_q=-1), _lib.MEA_ERR_SHAPE),
+    (dict(max_q=9), _lib.MEA_ERR_SHAPE),
+    (dict(hq=6, hkv=4), _lib.MEA_ERR_HEADS),
+    (dict(hkv=0), _lib.MEA_ERR_HEADS),
+    (dict(d=96), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=256), _lib.MEA_ERR_HEAD_DIM),
+    (dict(dtype=2), _lib.MEA_ERR_DTYPE),
+    (dict(mask=2), _lib.MEA_ERR_MASK),
+    (dict(scale=float("nan")), _lib.MEA_ERR_SCALE),
+    (dict(scale=float("inf")), _lib.MEA_ERR_SCALE),
+    (dict(q=A + 8), _lib.MEA_ERR_ALIGN),
+    (dict(out=A + 2), _lib.MEA_ERR_ALIGN),
+    (dict(lse=A + 2), _lib.MEA_ERR_ALIGN),
+])
+def test_forward_rejects(lib, kw, rc):
+    assert fwd(lib, **kw) == rc
+
+
+def dec(lib, **kw):
+    args = dict(q=A, k=A, v=A, out=A, lse=A, cu_k=A, n_seqs=2, total_k=100, max_k=60, hq=64,
+                hkv=8, d=128, scale=0.1, mask=1, slopes=None, dtype=1, ws=A, ws_bytes=1 << 30,
+                split=0, stream=None)
+    args.update(kw)
+    return lib.mea_decode_splitkv(args["q"], args["k"], args["v"], args["out"], args["lse"],
+                                  args["cu_k"], args["n_seqs"], args["total_k"], args["max_k"],
+                                  args["hq"], args["hkv"], args["d"], args["scale"],
+                                  args["mask"], args["slopes"], args["dtype"], args["ws"],
+                                  args["ws_bytes"], args["split"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,rc", [
+    (dict(k=None), _lib.MEA_ERR_NULL),
+    (dict(n_seqs=0), _lib.MEA_ERR_SHAPE),
+    (dict(max_k=101), _lib.MEA_ERR_SHAPE),
+    (dict(split=100), _lib.MEA_ERR_SHAPE),
+    (dict(hq=12, hkv=8), _lib.MEA_ERR_HEADS),
+    (dict(d=32), _lib.MEA_ERR_HEAD_DIM),
+    (dict(dtype=-1), _lib.MEA_ERR_DTYPE),
+    (dict(mask=3), _lib.MEA_ERR_MASK),
+    (dict(v=A + 4), _lib.MEA_ERR_ALIGN),
+])
+def test_decode_rejects(lib, kw, rc):
+    assert dec(lib, **kw) == rc
+
+
+def test_decode_workspace_size(lib):
+    # partials: (ceil(T_k / chunk) + n_seqs) slots x Hq x (D + 1) fp32, each region 256-aligned
+    n = lib.mea_decode_workspace_size(4, 1000, 16, 4, 128, 256)
+    slots = -(-1000 // 256) + 4
+    o = slots * 16 * 128 * 4
+    lse = slots * 16 * 4
+    assert n == -(-o // 256) * 256 + -(-lse // 256) * 256
+    assert lib.mea_decode_workspace_size(0, 10, 8, 8, 64, 0) == 0
+    assert lib.mea_decode_workspace_size(1, 10, 8, 8, 64, 65) == 0
+    assert lib.mea_decode_workspace_size(1, 10, 8, 3, 64, 64) == 0
+    # too small a workspace is rejected before any launch
+    need = lib.mea_decode_workspace_size(2, 100, 64, 8, 128, 64)
+    assert dec(lib, ws_bytes=need - 1, split=64) == _lib.MEA_ERR_WORKSPACE
+    assert dec(lib, ws=None, split=64) == _lib.MEA_ERR_WORKSPACE
+    assert dec(lib, ws=A + 16, split=64) == _lib.MEA_ERR_WORKSPACE
+
+
+def test_python_binding_fails_loudly_without_gpu():
+    import torch
+    import memory_efficient_attention_b200 as mea
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    q = torch.zeros((4, 2, 64), dtype=torch.float16)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    with pytest.raises(mea.MeaError):
+        mea.attention_packed(q, q, q, cu, cu, 4)
