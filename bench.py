@@ -450,8 +450,8 @@ def run_ours(args, world, rank, local):
     line["gpu_launches"] = launches_per_step * args.steps
     if e2e is not None:
         line["e2e"] = e2e
-    if not args.no_cpu_baseline and do_fwd:
-        sample, fl, desc = oracle_sample(1.5e11)
+    if not args.no_cpu_baseline and do_fwd and world == 1:
+        sample, fl, desc = oracle_sample(5.0e11)
         dt = time_oracle(sample)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
                                 "kind": "oracle", "sample": desc, "seconds": dt}
