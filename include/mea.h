@@ -59,7 +59,8 @@ typedef enum {
   MEA_ERR_CUDA = -9,          /* a CUDA runtime/driver call or a launch failed                */
   MEA_ERR_DEVICE_TIMEOUT = -10, /* a kernel gave up on a bounded wait (see mea_device_error)  */
   MEA_ERR_DEVICE = -11,       /* the current device is not an sm_100 part                     */
-  MEA_ERR_SCALE = -12         /* scale is not finite                                           */
+  MEA_ERR_SCALE = -12,        /* scale is not finite                                           */
+  MEA_ERR_SCRATCH_LIMIT = -13 /* the problem needs more scratch than the fixed static array    */
 } mea_status;
 
 typedef enum { MEA_F16 = 0, MEA_BF16 = 1 } mea_dtype;
@@ -118,6 +119,41 @@ int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, f
                        int n_heads_q, int n_heads_kv, int head_dim, float scale, int mask_kind,
                        const float* alibi_slopes, int dtype, void* workspace,
                        size_t workspace_bytes, int split_keys, void* stream);
+
+/*
+ * mea_decode_splitkv_noalloc — mea_decode_splitkv without a caller-provided workspace.
+ *
+ * The pages have no counterpart to this entry point: it exists for callers of the library, not
+ * for the method. Some callers cannot call cudaMalloc at all. For example, a plugin running
+ * inside a host runtime that has already reserved the device memory it will ever use and hands
+ * its plugins only their input and output tensors; or a latency-bound serving loop that must not
+ * pay for an allocation (and the device synchronisation an allocation can imply) on every decode
+ * step. This variant takes the same arguments as mea_decode_splitkv minus the workspace, and
+ * keeps the split-KV partials in a fixed array of MEA_DECODE_NOALLOC_SCRATCH_BYTES bytes that is
+ * part of the library itself (a file-scope __device__ array). Each GPU that loads the library
+ * holds that array until the process exits.
+ *
+ *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - The caller still provides q, k, v, out and (optionally) lse, as for mea_decode_splitkv.
+ *   - split_keys = 0 starts from the library's chunk size and doubles it until the partials fit
+ *     in the array; an explicit split_keys is used as given. If the partials
+ *     ((ceil(total_k / chunk) + n_seqs) * n_heads_q * (head_dim + 1) floats, each region rounded
+ *     up to 256 bytes) cannot fit, the call returns MEA_ERR_SCRATCH_LIMIT and launches nothing.
+ *   - The first call on a device looks up the array's device address on that device (one
+ *     cudaGetSymbolAddress, with that device current); make that first call before any stream
+ *     capture on that device.
+ *   - All calls share the one array and it keeps whatever the last call wrote. Nothing in it needs
+ *     to start at zero (every partial is written before it is read). Two calls whose kernels
+ *     overlap on the GPU (different streams, or different host threads, without ordering between
+ *     them) race on the array and give wrong results: order them on one stream or with events.
+ * Returns MEA_OK or a negative mea_status, like mea_decode_splitkv.
+ */
+#define MEA_DECODE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                               const int32_t* cu_seqlens_k, int n_seqs, int total_k,
+                               int max_seqlen_k, int n_heads_q, int n_heads_kv, int head_dim,
+                               float scale, int mask_kind, const float* alibi_slopes, int dtype,
+                               int split_keys, void* stream);
 
 /* mea_status_string — a static English description of a mea_status value. */
 const char* mea_status_string(int status);

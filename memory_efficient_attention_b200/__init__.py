@@ -25,7 +25,7 @@ from . import _lib
 from ._lib import MeaError  # noqa: F401
 
 __all__ = [
-    "memory_efficient_attention", "attention_packed", "decode_splitkv",
+    "memory_efficient_attention", "attention_packed", "decode_splitkv", "decode_splitkv_noalloc",
     "decode_workspace_size", "alibi_slopes", "BlockDiagonalMask", "BlockDiagonalCausalMask",
     "LowerTriangularMask", "device_error", "set_wait_timeout_ns", "MeaError", "library_path",
 ]
@@ -136,6 +136,31 @@ def decode_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
         _dtype_code(q.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(),
         int(split_keys), _stream(q.device))
     _lib.check(rc, "mea_decode_splitkv")
+    return out, lse
+
+
+def decode_splitkv_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                           cu_seqlens_k: torch.Tensor, max_seqlen_k: int, out: torch.Tensor,
+                           lse: Optional[torch.Tensor] = None,
+                           alibi_slopes: Optional[torch.Tensor] = None,
+                           scale: Optional[float] = None, split_keys: int = 0):
+    """:func:`decode_splitkv` for callers that cannot allocate device memory.
+
+    The split-KV partials go to a fixed array inside the library instead of a workspace, so this
+    call performs no device allocation of its own: the caller passes the output buffers (``out``
+    ``[B, Hq, D]``, optional ``lse`` ``[Hq, B]`` fp32) along with the inputs. Calls that overlap on
+    the GPU share that array and race; keep them ordered on one stream. Raises ``MeaError`` with
+    ``MEA_ERR_SCRATCH_LIMIT`` when the partials cannot fit in the array.
+    """
+    b, hq, d = q.shape
+    tk, hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = _lib.load().mea_decode_splitkv_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_k), b, tk,
+        int(max_seqlen_k), hq, hkv, d, float(scale), _lib.MEA_MASK_CAUSAL, _ptr(alibi_slopes),
+        _dtype_code(q.dtype), int(split_keys), _stream(q.device))
+    _lib.check(rc, "mea_decode_splitkv_noalloc")
     return out, lse
 
 

@@ -21,6 +21,7 @@ MEA_ERR_CUDA = -9
 MEA_ERR_DEVICE_TIMEOUT = -10
 MEA_ERR_DEVICE = -11
 MEA_ERR_SCALE = -12
+MEA_ERR_SCRATCH_LIMIT = -13
 
 MEA_F16 = 0
 MEA_BF16 = 1
@@ -28,7 +29,8 @@ MEA_MASK_NONE = 0
 MEA_MASK_CAUSAL = 1
 
 EXPORTS = ("mea_forward", "mea_decode_workspace_size", "mea_decode_splitkv",
-           "mea_status_string", "mea_device_error", "mea_set_wait_timeout_ns", "mea_version")
+           "mea_decode_splitkv_noalloc", "mea_status_string", "mea_device_error",
+           "mea_set_wait_timeout_ns", "mea_version")
 
 _lib = None
 
@@ -51,6 +53,9 @@ def load() -> ctypes.CDLL:
     lib.mea_decode_splitkv.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp,
                                        ci, vp, sz, ci, vp]
     lib.mea_decode_splitkv.restype = ci
+    lib.mea_decode_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf,
+                                               ci, vp, ci, ci, vp]
+    lib.mea_decode_splitkv_noalloc.restype = ci
     lib.mea_status_string.argtypes = [ci]
     lib.mea_status_string.restype = ctypes.c_char_p
     lib.mea_device_error.argtypes = [ctypes.POINTER(ci), ci]

@@ -186,6 +186,37 @@ bool dec_layout(int n_seqs, int total_k, int hq, int hkv, int d, int split_keys,
 
 }  // namespace
 
+// ------------------------------------------------------------------------------------------
+// Fixed scratch for mea_decode_splitkv_noalloc: the split-KV partials live in this array, which
+// belongs to the library image (every GPU that loads the library holds it until exit), so that
+// callers which cannot allocate device memory can still decode. Host code must not pass the
+// symbol itself to a kernel: on the host it is only a stand-in; its device address is looked up
+// once per device with cudaGetSymbolAddress.
+// ------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char mea_noalloc_scratch[MEA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+void* g_noalloc_addr[kMaxDevices] = {};
+cudaError_t g_noalloc_err[kMaxDevices] = {};
+std::once_flag g_noalloc_once[kMaxDevices];
+
+// Device address of mea_noalloc_scratch on the current device (looked up on first use).
+int noalloc_scratch_address(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MEA_ERR_CUDA;
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, mea_noalloc_scratch);
+    g_noalloc_addr[dev] = p;
+  });
+  if (g_noalloc_err[dev] != cudaSuccess || g_noalloc_addr[dev] == nullptr) return MEA_ERR_CUDA;
+  *ptr = g_noalloc_addr[dev];
+  return MEA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* mea_version(void) { return "mea 0.1.0 (sm_100a)"; }
@@ -205,6 +236,10 @@ const char* mea_status_string(int status) {
     case MEA_ERR_DEVICE_TIMEOUT: return "MEA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
     case MEA_ERR_DEVICE: return "MEA_ERR_DEVICE: the current device is not sm_100";
     case MEA_ERR_SCALE: return "MEA_ERR_SCALE: scale must be finite";
+    case MEA_ERR_SCRATCH_LIMIT:
+      return "MEA_ERR_SCRATCH_LIMIT: the decode partials do not fit in the library's fixed "
+             "scratch array (MEA_DECODE_NOALLOC_SCRATCH_BYTES); use mea_decode_splitkv with a "
+             "workspace, or a larger split_keys";
     default: return "unknown mea_status";
   }
 }
@@ -331,6 +366,84 @@ int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, f
   p.slopes = alibi_slopes;
   p.ws_o = static_cast<float*>(workspace);
   p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.lse_off);
+  p.n_seqs = n_seqs;
+  p.hq = n_heads_q;
+  p.R = R;
+  p.RB = decode_rb(R);
+  p.n_hb = n_heads_q / p.RB;
+  p.chunk = L.chunk;
+  p.n_slots = L.n_slots;
+  p.n_items = static_cast<long long>(L.n_slots) * p.n_hb;
+  p.c1 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+
+  CUtensorMap tk, tv;
+  const uint64_t tk_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
+  if (!encode_3d(&tk, k, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 64) ||
+      !encode_3d(&tv, v, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 64))
+    return MEA_ERR_CUDA;
+  const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool alibi = alibi_slopes != nullptr;
+  if (head_dim == 128)
+    return dtype == MEA_BF16 ? launch_dec_d<128, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+                             : launch_dec_d<128, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
+  return dtype == MEA_BF16 ? launch_dec_d<64, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+                           : launch_dec_d<64, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
+}
+
+int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                               const int32_t* cu_seqlens_k, int n_seqs, int total_k,
+                               int max_seqlen_k, int n_heads_q, int n_heads_kv, int head_dim,
+                               float scale, int mask_kind, const float* alibi_slopes, int dtype,
+                               int split_keys, void* stream) {
+  if (!q || !k || !v || !out || !cu_seqlens_k) return MEA_ERR_NULL;
+  if (n_seqs < 1 || total_k < 0 || max_seqlen_k < 0 || max_seqlen_k > total_k)
+    return MEA_ERR_SHAPE;
+  if (split_keys < 0 || split_keys % 64) return MEA_ERR_SHAPE;
+  if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
+  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
+  if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
+  if (!std::isfinite(scale)) return MEA_ERR_SCALE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)) || !aligned(cu_seqlens_k, 4) ||
+      (alibi_slopes && !aligned(alibi_slopes, 4)))
+    return MEA_ERR_ALIGN;
+
+  // Chunk size: as given, or the library's choice doubled until the partials fit the array.
+  const size_t limit = MEA_DECODE_NOALLOC_SCRATCH_BYTES;
+  DecLayout L;
+  DeviceInfo di;
+  if (split_keys != 0) {
+    if (!dec_layout(n_seqs, total_k, n_heads_q, n_heads_kv, head_dim, split_keys, 0, L))
+      return MEA_ERR_SHAPE;
+    if (L.total > limit) return MEA_ERR_SCRATCH_LIMIT;
+    if (int rc = current_device_info(di); rc != MEA_OK) return rc;
+  } else {
+    if (int rc = current_device_info(di); rc != MEA_OK) return rc;
+    if (!dec_layout(n_seqs, total_k, n_heads_q, n_heads_kv, head_dim, 0, di.sms, L))
+      return MEA_ERR_SHAPE;
+    int chunk = L.chunk;
+    while (L.total > limit && chunk < (1 << 24) && chunk < total_k) {
+      chunk *= 2;
+      if (!dec_layout(n_seqs, total_k, n_heads_q, n_heads_kv, head_dim, chunk, 0, L))
+        return MEA_ERR_SHAPE;
+    }
+    if (L.total > limit) return MEA_ERR_SCRATCH_LIMIT;
+  }
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch_address(&scratch); rc != MEA_OK) return rc;
+
+  const int R = n_heads_q / n_heads_kv;
+  mea::DecParams p{};
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.cu_k = cu_seqlens_k;
+  p.slopes = alibi_slopes;
+  p.ws_o = static_cast<float*>(scratch);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(scratch) + L.lse_off);
   p.n_seqs = n_seqs;
   p.hq = n_heads_q;
   p.R = R;
