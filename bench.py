@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--decode-requests", type=int, default=64,
+                    help="use only the first N requests of the decode workload (profiling)")
     return ap.parse_args()
 
 
@@ -280,7 +282,7 @@ def run_ours(args, world, rank, local):
     # ---- decode inputs
     if do_dec:
         g.manual_seed(w4.seed)
-        lk = w4.seqlens_k
+        lk = w4.seqlens_k[:max(1, args.decode_requests)]
         tk = sum(lk)
         n_req = len(lk)
         dq = torch.randn((n_req, 64, 128), generator=g, device=dev, dtype=torch.float32).bfloat16()
@@ -418,7 +420,8 @@ def run_ours(args, world, rank, local):
                         f"{w2.total_q} tokens in {len(w2.seqlens_q)} segments U[64,4096]) + "
                         "split-KV decode (bf16, 64 requests x 1 token, KV U[512,32768], "
                         "64 q / 8 kv heads, D=128)"),
-           "prefill_seqlens": w2.seqlens_q, "decode_total_kv_tokens": w4.total_k,
+           "prefill_seqlens": w2.seqlens_q,
+           "decode_total_kv_tokens": sum(w4.seqlens_k[:max(1, args.decode_requests)]),
            "l2": "inputs larger than L2 (q 268 MB; K+V 4.3 GB), no flush",
            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
     line["config"] = cfg

@@ -1,28 +1,34 @@
 // fwd_sm100.cuh — persistent, warp-specialised forward kernel of exact attention for sm_100a.
 //
-// Computes, for every (segment, 128-row query tile, head block), out = softmax(QK^T*scale+bias)V
+// Computes, for every (segment, query-tile pair, head block), out = softmax(QK^T*scale+bias)V
 // and lse, one 128-key tile at a time with an online softmax, so the score matrix only ever
 // lives in tensor memory (the blockwise engine of "大模型推理加速终极指南", section 1; masks and
 // bias of "How to Build Memory-Efficient Transformers with xFormers…", techniques 1, 3 and 5).
 //
-// Roles (192 threads, one CTA per SM):
-//   warps 0-3  softmax / correction / epilogue: thread r owns row r of the tile = TMEM lane r.
-//   warp 4     TMA producer: Q tile once per work item, then K_j, V_j through an NS-slot ring.
-//   warp 5     tcgen05 issuer (one lane): S_j = Q K_j^T into TMEM buffer j%2, O += P_j V_j with
-//              P_j read from TMEM (written over S_j by the softmax warps). Also owns TMEM.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D). P_j is bf16/f16-packed in the first 64
-// columns of its S buffer.
+// A work item is a pair of 128-row query sub-tiles (h = 0, 1) that share every K/V tile.
+// Roles (384 threads, one CTA per SM; warps 10-11 only lend their registers):
+//   warps 0-3  softmax / correction / epilogue of sub-tile 0: thread r owns row r = TMEM lane r.
+//   warps 4-7  the same for sub-tile 1.
+//   warp 8     tcgen05 issuer (one lane); also allocates TMEM. Per K/V tile j it issues
+//              PV_0(j-1), QK_0(j), PV_1(j-1), QK_1(j): while one warpgroup turns S_h(j) into
+//              P_h(j), the tensor core works on the other sub-tile, and when S_h(j) is ready the
+//              earlier PV_h(j-1) has completed, so O_h can be rescaled without another wait.
+//   warp 9     TMA producer: both Q sub-tiles once per item, then K_j, V_j through an NS-slot ring.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256, 256+D), O_1 [256+D, 256+2D). P_h(j) is
+// written bf16/f16-packed over the first 64 columns of S_h and read from there as the A operand.
 //
-// GQA packing: a 128-row tile holds 128/P tokens x P query heads of one KV group (row r ->
-// token tok0 + r/P, head hb*P + r%P), loaded by one 3-D TMA box [128/P tokens, P heads, 64 d],
-// so each K/V tile is read once for the P heads that share it.
+// GQA packing: a 128-row sub-tile holds 128/P tokens x P query heads of one KV group (row r ->
+// token tok0 + h*128/P + r/P, head hb*P + r%P), loaded by one 3-D TMA box [128/P tokens, P heads,
+// 64 d], so each K/V tile is read once for the 2P heads/2*128/P tokens that share it.
 //
-// Work items (tile, segment, head block) are visited round-robin by the persistent CTAs in
-// heavy-first order for causal masks (the last query tiles have the most keys).
+// Work items (pair, segment, head block) are visited round-robin by the persistent CTAs in
+// heavy-first order for causal masks (the last query tiles of a segment have the most keys).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <type_traits>
 
 #include "ptx.cuh"
 
@@ -38,10 +44,10 @@ struct FwdParams {
   int total_q;
   int hq;
   int n_hb;          // head blocks = hq / P
-  int P;             // query heads packed per tile (a power of two dividing R)
+  int P;             // query heads packed per sub-tile (a power of two dividing R)
   int R;             // query heads per KV head
-  int tok_per_tile;  // 128 / P
-  int t_max;         // max query tiles of a segment
+  int tok_per_tile;  // 128 / P tokens per sub-tile
+  int t_max;         // max sub-tile pairs of a segment
   long long n_items; // t_max * n_seqs * n_hb
   float c1;          // scale * log2(e)
   unsigned long long timeout_ns;
@@ -54,18 +60,24 @@ struct FwdCfg {
   static constexpr int ATOMS = D / 64;  // 128-byte swizzle atoms along the head dim
   static constexpr uint32_t ATOM_BYTES = 128 * 128;
   static constexpr uint32_t TILE_BYTES = 128 * D * 2;
-  static constexpr int NS = (D == 128) ? 6 : 8;
-  static constexpr uint32_t SMEM_Q = 0;
-  static constexpr uint32_t SMEM_KV = TILE_BYTES;
+  static constexpr int NS = (D == 128) ? 5 : 8;
+  static constexpr uint32_t SMEM_Q = 0;                 // two Q sub-tiles
+  static constexpr uint32_t SMEM_KV = 2 * TILE_BYTES;
   static constexpr uint32_t SMEM_BAR = SMEM_KV + NS * TILE_BYTES;
   static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 384;
+  // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); warps 8-11
+  // give theirs down to REGS_OTHER so that the two softmax warpgroups can take REGS_SOFTMAX.
+  // 256 * REGS_SOFTMAX + 128 * REGS_OTHER must not exceed 64512.
+  static constexpr int REGS_SOFTMAX = 216;
+  static constexpr int REGS_OTHER = 64;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t TM_O = 256;
+  static constexpr uint32_t TM_O = 256;                 // O_h at TM_O + h*D
 };
 
 struct FwdItem {
-  int seg, hb, q0, lq, k0, lk, tok0, n_kv;
+  int seg, hb, q0, lq, k0, lk, tok0;
+  int n_kv[2];
   bool live;
 };
 
@@ -81,16 +93,24 @@ __device__ __forceinline__ FwdItem fwd_decode_item(const FwdParams& p, long long
   it.lq = __ldg(p.cu_q + it.seg + 1) - it.q0;
   it.k0 = __ldg(p.cu_k + it.seg);
   it.lk = __ldg(p.cu_k + it.seg + 1) - it.k0;
-  const int nt = (it.lq + p.tok_per_tile - 1) / p.tok_per_tile;
+  const int tpp = 2 * p.tok_per_tile;
+  const int np = (it.lq + tpp - 1) / tpp;
   const int t = causal ? (p.t_max - 1 - tr) : tr;
-  it.live = (t >= 0) && (t < nt);
-  it.tok0 = t * p.tok_per_tile;
-  int kv_end = it.lk;
-  if (causal) {
-    const int last = min(it.tok0 + p.tok_per_tile, it.lq) - 1;
-    kv_end = min(it.lk, last + 1 + it.lk - it.lq);
+  it.live = (t >= 0) && (t < np);
+  it.tok0 = t * tpp;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int first = it.tok0 + h * p.tok_per_tile;
+    int kv_end = 0;
+    if (first < it.lq) {
+      kv_end = it.lk;
+      if (causal) {
+        const int last = min(first + p.tok_per_tile, it.lq) - 1;
+        kv_end = min(it.lk, last + 1 + it.lk - it.lq);
+      }
+    }
+    it.n_kv[h] = kv_end > 0 ? (kv_end + 127) / 128 : 0;
   }
-  it.n_kv = kv_end > 0 ? (kv_end + 127) / 128 : 0;
   return it;
 }
 
@@ -105,8 +125,20 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   }
 }
 
+// End of a role: every thread of the CTA arrives here (from its own code path) before the
+// tcgen05 issuer warp releases tensor memory.
+__device__ __forceinline__ void fwd_teardown(bool owner, uint32_t tmem, uint32_t ncols) {
+  tc_fence_before();
+  asm volatile("bar.sync 0;" ::: "memory");
+  if (owner) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, ncols);
+  }
+}
+
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
     mea_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -119,7 +151,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t kv_s0 = sbase + C::SMEM_KV;
 
   constexpr int B_QF = 0, B_QE = 1, B_KVF = 2, B_KVE = 2 + C::NS, B_SF = 2 + 2 * C::NS;
-  constexpr int B_PF = B_SF + 2, B_OD = B_PF + 2, B_OE = B_OD + 1, B_DR = B_OE + 1;
+  constexpr int B_PF = B_SF + 2, B_OF = B_PF + 2, B_OE = B_OF + 2, B_DR = B_OE + 2;
   constexpr int N_BARS = B_DR + 1;
   const uint32_t bar0 = sbase + C::SMEM_BAR;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
@@ -138,22 +170,22 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(BAR(B_KVF + s), 1);
       mbar_init(BAR(B_KVE + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(BAR(B_SF + b), 1);
-      mbar_init(BAR(B_PF + b), 128);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(BAR(B_SF + h), 1);
+      mbar_init(BAR(B_PF + h), 128);
+      mbar_init(BAR(B_OF + h), 1);
+      mbar_init(BAR(B_OE + h), 128);
     }
-    mbar_init(BAR(B_OD), 1);
-    mbar_init(BAR(B_OE), 128);
     mbar_init(BAR(B_DR), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 9 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 5) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -162,24 +194,30 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  static_assert(256 * C::REGS_SOFTMAX + 128 * C::REGS_OTHER <= 384 * 168, "register split");
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
+    if (warp == 9) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       uint32_t kv_cnt = 0, q_cnt = 0;
       bool ok = true;
       for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
         const FwdItem it = fwd_decode_item(p, lin, CAUSAL);
-        if (!it.live || it.n_kv == 0) continue;
+        const int nmax = max(it.n_kv[0], it.n_kv[1]);
+        if (!it.live || nmax == 0) continue;
         const int g = (it.hb * p.P) / p.R;
         ok = mbar_wait(BAR(B_QE), (q_cnt & 1u) ^ 1u, abort_flag, tmo, ecode | 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(BAR(B_QF), C::TILE_BYTES);
+        mbar_arrive_expect_tx(BAR(B_QF), 2 * C::TILE_BYTES);
 #pragma unroll
-        for (int a = 0; a < C::ATOMS; ++a)
-          tma_load_3d(q_s + a * C::ATOM_BYTES, &tm_q, BAR(B_QF), a * 64, it.hb * p.P,
-                      it.q0 + it.tok0);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int a = 0; a < C::ATOMS; ++a)
+            tma_load_3d(q_s + h * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_q, BAR(B_QF), a * 64,
+                        it.hb * p.P, it.q0 + it.tok0 + h * p.tok_per_tile);
         ++q_cnt;
-        for (int j = 0; j < it.n_kv && ok; ++j) {
+        for (int j = 0; j < nmax && ok; ++j) {
 #pragma unroll 1
           for (int w = 0; w < 2; ++w) {
             const uint32_t s = kv_cnt % C::NS;
@@ -209,106 +247,115 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
-  } else if (warp == 5) {
+    } else if (warp == 8) {
     // ---------------------------------------------------------------- tcgen05 issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = umma_idesc_f16(BF16, 128, 128, false, false);
       constexpr uint32_t IDESC_PV = umma_idesc_f16(BF16, 128, D, false, true);
-      uint32_t kv_cnt = 0, q_cnt = 0, tile = 0, items_pv = 0;
+      uint32_t kv_cnt = 0, q_cnt = 0;
+      uint32_t pv_cnt[2] = {0, 0}, oe_cnt[2] = {0, 0};
       bool ok = true;
-      bool pend_valid = false, pend_first = false;
-      uint32_t pend_tile = 0, pend_vslot = 0, pend_vph = 0;
-
-      auto issue_pv = [&]() -> bool {
-        const uint32_t b = pend_tile & 1u;
-        if (!mbar_wait(BAR(B_PF + b), (pend_tile >> 1) & 1u, abort_flag, tmo, ecode | 3))
-          return false;
-        if (pend_first) {
-          if (!mbar_wait(BAR(B_OE), (items_pv & 1u) ^ 1u, abort_flag, tmo, ecode | 4))
-            return false;
-          ++items_pv;
-        }
-        if (!mbar_wait(BAR(B_KVF + pend_vslot), pend_vph, abort_flag, tmo, ecode | 5))
-          return false;
-        tc_fence_after();
-        const uint32_t vbase = kv_s0 + pend_vslot * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint64_t bd = umma_desc_sw128(vbase + kk * 2048, C::ATOM_BYTES, 1024);
-          mma_ts(tmem + C::TM_O, tmem + b * 128 + kk * 8, bd, IDESC_PV,
-                 (pend_first && kk == 0) ? 0u : 1u);
-        }
-        mma_commit(BAR(B_KVE + pend_vslot));
-        mma_commit(BAR(B_OD));
-        return true;
-      };
-
       for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
         const FwdItem it = fwd_decode_item(p, lin, CAUSAL);
-        if (!it.live || it.n_kv == 0) continue;
+        const int nmax = max(it.n_kv[0], it.n_kv[1]);
+        if (!it.live || nmax == 0) continue;
         ok = mbar_wait(BAR(B_QF), q_cnt & 1u, abort_flag, tmo, ecode | 6);
         if (!ok) break;
         tc_fence_after();
-        for (int j = 0; j < it.n_kv; ++j) {
-          const uint32_t s = kv_cnt % C::NS;
-          const uint32_t ph = (kv_cnt / C::NS) & 1u;
-          ok = mbar_wait(BAR(B_KVF + s), ph, abort_flag, tmo, ecode | 7);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t b = tile & 1u;
-          const uint32_t kbase = kv_s0 + s * C::TILE_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-            const uint64_t ad = umma_desc_sw128(q_s + off, 16, 1024);
-            const uint64_t bd = umma_desc_sw128(kbase + off, 16, 1024);
-            mma_ss(tmem + b * 128, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(BAR(B_SF + b));
-          mma_commit(BAR(B_KVE + s));
-          if (j == it.n_kv - 1) mma_commit(BAR(B_QE));
-          ++kv_cnt;
-          const uint32_t vs = kv_cnt % C::NS;
-          const uint32_t vph = (kv_cnt / C::NS) & 1u;
-          ++kv_cnt;
-          if (pend_valid) {
-            ok = issue_pv();
+        const uint32_t base = kv_cnt;
+        for (int j = 0; j <= nmax && ok; ++j) {
+          const uint32_t ks = (base + 2 * j) % C::NS;
+          const uint32_t vs = (base + 2 * j - 1) % C::NS;  // slot of V_{j-1} (j >= 1)
+          if (j < nmax) {
+            ok = mbar_wait(BAR(B_KVF + ks), ((base + 2 * j) / C::NS) & 1u, abort_flag, tmo,
+                           ecode | 7);
             if (!ok) break;
+            tc_fence_after();
           }
-          pend_valid = true;
-          pend_first = (j == 0);
-          pend_tile = tile;
-          pend_vslot = vs;
-          pend_vph = vph;
-          ++tile;
+          bool v_ready = false;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int nh = it.n_kv[h];
+            if (j >= 1 && j <= nh) {
+              // ---- O_h += P_h(j-1) V_{j-1}
+              if (!v_ready) {
+                ok = mbar_wait(BAR(B_KVF + vs), ((base + 2 * j - 1) / C::NS) & 1u, abort_flag,
+                               tmo, ecode | 5);
+                if (!ok) break;
+                v_ready = true;
+              }
+              ok = mbar_wait(BAR(B_PF + h), pv_cnt[h] & 1u, abort_flag, tmo, ecode | 3);
+              if (!ok) break;
+              if (j == 1) {
+                ok = mbar_wait(BAR(B_OE + h), (oe_cnt[h] & 1u) ^ 1u, abort_flag, tmo, ecode | 4);
+                if (!ok) break;
+                ++oe_cnt[h];
+              }
+              tc_fence_after();
+              const uint32_t vbase = kv_s0 + vs * C::TILE_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < C::BN / 16; ++kk) {
+                const uint64_t bd = umma_desc_sw128(vbase + kk * 2048, C::ATOM_BYTES, 1024);
+                mma_ts(tmem + C::TM_O + h * D, tmem + h * 128 + kk * 8, bd, IDESC_PV,
+                       (j == 1 && kk == 0) ? 0u : 1u);
+              }
+              ++pv_cnt[h];
+              if (j == nh) mma_commit(BAR(B_OF + h));
+            }
+            if (j < nh) {
+              // ---- S_h = Q_h K_j^T
+              const uint32_t kbase = kv_s0 + ks * C::TILE_BYTES;
+              const uint32_t qbase = q_s + h * C::TILE_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+                const uint64_t ad = umma_desc_sw128(qbase + off, 16, 1024);
+                const uint64_t bd = umma_desc_sw128(kbase + off, 16, 1024);
+                mma_ss(tmem + h * 128, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(BAR(B_SF + h));
+            }
+          }
+          if (!ok) break;
+          if (j < nmax) mma_commit(BAR(B_KVE + ks));
+          if (j >= 1) mma_commit(BAR(B_KVE + vs));
+          if (j == nmax - 1) mma_commit(BAR(B_QE));
         }
         if (!ok) break;
+        kv_cnt = base + 2 * nmax;
         ++q_cnt;
       }
-      if (ok && pend_valid) ok = issue_pv();
       // Every MMA issued so far must finish before TMEM is released.
       mma_commit(BAR(B_DR));
       volatile int never = 0;
       mbar_wait(BAR(B_DR), 0, &never, tmo, ecode | 14);
     }
+    }
+    fwd_teardown(warp == 8, tmem, C::TMEM_COLS);
   } else {
-    // ---------------------------------------------------------------- softmax warps 0-3
-    const int r = threadIdx.x;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int h = warp >> 2;           // sub-tile of this warpgroup
+    const int r = threadIdx.x & 127;   // row within the sub-tile = TMEM lane
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t t_s = t_lane + h * 128;
+    const uint32_t t_o = t_lane + C::TM_O + h * D;
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr float LN2 = 0.6931471805599453f;
-    uint32_t tile = 0;
+    uint32_t tile = 0, ocnt = 0;
     bool ok = true;
     for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
       const FwdItem it = fwd_decode_item(p, lin, CAUSAL);
       if (!it.live) continue;
-      const int tok = it.tok0 + r / p.P;
+      const int sub0 = it.tok0 + h * p.tok_per_tile;  // first token of this sub-tile
+      const int tok = sub0 + r / p.P;
       const int head = it.hb * p.P + (r % p.P);
       const bool row_valid = tok < it.lq;
+      const int nh = it.n_kv[h];
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       OutT* orow = reinterpret_cast<OutT*>(p.out) +
                    (static_cast<size_t>(it.q0 + tok) * p.hq + head) * D;
-      if (it.n_kv == 0) {
+      if (nh == 0) {
         if (row_valid) {
           uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -317,37 +364,91 @@ __global__ void __launch_bounds__(192, 1)
         }
         continue;
       }
-      const int pos = tok + it.lk - it.lq;       // key position of this query row
-      const int p_min = it.tok0 + it.lk - it.lq;  // position of the tile's first row
+      const int pos = tok + it.lk - it.lq;      // key position of this query row
+      const int p_min = sub0 + it.lk - it.lq;   // position of the sub-tile's first row
       float slope2 = 0.f;
       if constexpr (ALIBI) slope2 = __ldg(p.slopes + head) * LOG2E;
       float m_ref = -INFINITY, l = 0.f;
-      for (int j = 0; j < it.n_kv; ++j) {
-        const uint32_t b = tile & 1u;
-        ok = mbar_wait(BAR(B_SF + b), (tile >> 1) & 1u, abort_flag, tmo, ecode | 8);
+      for (int j = 0; j < nh; ++j) {
+        ok = mbar_wait(BAR(B_SF + h), tile & 1u, abort_flag, tmo, ecode | 8);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
         uint32_t sr[128];
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
-          tmem_ld32(t_lane + b * 128 + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c4 * 32]));
+          tmem_ld32(t_s + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c4 * 32]));
         tmem_wait_ld();
         const int kv0 = j * 128;
         const bool need_mask = (kv0 + 128 > it.lk) || (CAUSAL && kv0 + 127 > p_min);
         const int limit = (CAUSAL ? min(pos, it.lk - 1) : it.lk - 1) - kv0;
-        const float dd0 = static_cast<float>(kv0 - pos);
         float x[128];
-        float mt = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float v = __uint_as_float(sr[c]) * p.c1;
-          if constexpr (ALIBI) v = fmaf(-slope2, fabsf(dd0 + static_cast<float>(c)), v);
-          if (need_mask && c > limit) v = -INFINITY;
-          x[c] = v;
-          mt = fmaxf(mt, v);
+        for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+        // Row maximum of this tile (log2 units) and the exponent offset for this tile:
+        //   fast path, no ALiBi:      x = S (raw), score = c1*x,        p = 2^(c1*x - m_ref)
+        //   fast path, causal ALiBi:  x = c1*S + slope2*c, score = x + K with the row/tile
+        //                             constant K = slope2*(kv0 - pos), p = 2^(x - (m_ref - K))
+        //   general path:             x = score,                        p = 2^(x - m_ref)
+        const bool fast = (p.c1 > 0.f) && (!ALIBI || CAUSAL);
+        float m_tile, kconst = 0.f;
+        if (fast) {
+          if constexpr (ALIBI) {
+            const uint64_t c1x2 = f2_pack(p.c1, p.c1);
+            const uint64_t inc = f2_pack(2.f * slope2, 2.f * slope2);
+#pragma unroll
+            for (int c32 = 0; c32 < 4; ++c32) {
+              uint64_t cb = f2_pack(slope2 * static_cast<float>(c32 * 32),
+                                    slope2 * static_cast<float>(c32 * 32 + 1));
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int c = c32 * 32 + 2 * i;
+                f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), c1x2, cb), x[c], x[c + 1]);
+                cb = f2_add(cb, inc);
+              }
+            }
+            kconst = slope2 * static_cast<float>(kv0 - pos);
+          }
+          if (need_mask) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c > limit) x[c] = -INFINITY;
+          }
+          float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+#pragma unroll
+          for (int i = 0; i < 15; ++i) {
+            a0 = max3f(a0, x[8 + 8 * i + 0], x[8 + 8 * i + 1]);
+            a1 = max3f(a1, x[8 + 8 * i + 2], x[8 + 8 * i + 3]);
+            a2 = max3f(a2, x[8 + 8 * i + 4], x[8 + 8 * i + 5]);
+            a3 = max3f(a3, x[8 + 8 * i + 6], x[8 + 8 * i + 7]);
+          }
+          a0 = max3f(a0, x[4], x[5]);
+          a1 = max3f(a1, x[6], x[7]);
+          const float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+          if constexpr (ALIBI)
+            m_tile = mx + kconst;
+          else
+            m_tile = mx * p.c1;
+        } else {
+          const float dd0 = static_cast<float>(kv0 - pos);
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            float v = x[c] * p.c1;
+            if constexpr (ALIBI) v = fmaf(-slope2, fabsf(dd0 + static_cast<float>(c)), v);
+            if (need_mask && c > limit) v = -INFINITY;
+            x[c] = v;
+          }
+          float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+#pragma unroll
+          for (int i = 0; i < 31; ++i) {
+            a0 = fmaxf(a0, x[4 + 4 * i + 0]);
+            a1 = fmaxf(a1, x[4 + 4 * i + 1]);
+            a2 = fmaxf(a2, x[4 + 4 * i + 2]);
+            a3 = fmaxf(a3, x[4 + 4 * i + 3]);
+          }
+          m_tile = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
         }
-        const float m_new = fmaxf(m_ref, mt);
+        const float m_new = fmaxf(m_ref, m_tile);
         const bool resc = m_new > m_ref + 8.0f;
         float alpha = 1.f;
         if (resc) {
@@ -356,56 +457,63 @@ __global__ void __launch_bounds__(192, 1)
           m_ref = m_new;
         }
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float rs = 0.f;
+        // p = 2^(mul*x - off) on pairs, summed in four independent pair accumulators
+        const float mul = (fast && !ALIBI) ? p.c1 : 1.f;
+        const float off = m_use - kconst;
+        const uint64_t mulx2 = f2_pack(mul, mul);
+        const uint64_t negoff = f2_pack(-off, -off);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2_approx(x[c4 * 32 + 2 * i] - m_use);
-            const float p1 = ex2_approx(x[c4 * 32 + 2 * i + 1] - m_use);
-            rs += p0 + p1;
+            const uint64_t e =
+                f2_fma(f2_pack(x[c4 * 32 + 2 * i], x[c4 * 32 + 2 * i + 1]), mulx2, negoff);
+            float e0, e1;
+            f2_unpack(e, e0, e1);
+            const float p0 = ex2_approx(e0);
+            const float p1 = ex2_approx(e1);
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
             pk[i] = pack2<BF16>(p0, p1);
           }
-          tmem_st16(t_lane + b * 128 + c4 * 16, pk);
+          tmem_st16(t_s + c4 * 16, pk);
         }
-        l += rs;
-        tmem_wait_st();
-        if (j > 0) {
-          // O += P_{j-1} V_{j-1} must be complete before O is rescaled (and is waited on once
-          // per tile in order, so the barrier phases are never skipped).
-          ok = mbar_wait(BAR(B_OD), (tile - 1) & 1u, abort_flag, tmo, ecode | 9);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          if (__any_sync(0xffffffffu, resc)) {
-            tc_fence_after();
+        {
+          const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          float r0, r1;
+          f2_unpack(t, r0, r1);
+          l += r0 + r1;
+        }
+        // O_h holds tiles < j and its last PV has completed (it was issued before QK_h(j)).
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-            for (int c4 = 0; c4 < D / 32; ++c4) {
-              uint32_t o[32];
-              tmem_ld32(t_lane + C::TM_O + c4 * 32, o);
-              tmem_wait_ld();
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c4 * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(t_lane + C::TM_O + c4 * 32, o);
-            }
-            tmem_wait_st();
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + c4 * 32, o);
           }
         }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(B_PF + b));
+        mbar_arrive(BAR(B_PF + h));
         ++tile;
       }
       if (!ok) break;
       // ---- epilogue: O / l -> out, lse
-      ok = mbar_wait(BAR(B_OD), (tile - 1) & 1u, abort_flag, tmo, ecode | 10);
+      ok = mbar_wait(BAR(B_OF + h), ocnt & 1u, abort_flag, tmo, ecode | 10);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
+      ++ocnt;
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t o[32];
-        tmem_ld32(t_lane + C::TM_O + c4 * 32, o);
+        tmem_ld32(t_o + c4 * 32, o);
         tmem_wait_ld();
         if (row_valid) {
           uint32_t pk[16];
@@ -420,20 +528,14 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(BAR(B_OE));
+      mbar_arrive(BAR(B_OE + h));
       if (row_valid && p.lse)
         p.lse[static_cast<size_t>(head) * p.total_q + it.q0 + tok] =
             l > 0.f ? (m_ref + __log2f(l)) * LN2 : -INFINITY;
     }
+    fwd_teardown(false, tmem, C::TMEM_COLS);
   }
 #undef BAR
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 5) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
 }
 
 }  // namespace mea

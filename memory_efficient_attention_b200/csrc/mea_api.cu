@@ -295,7 +295,7 @@ int mea_forward(const void* q, const void* k, const void* v, void* out, float* l
   p.R = R;
   p.n_hb = n_heads_q / P;
   p.tok_per_tile = 128 / P;
-  p.t_max = (max_seqlen_q + p.tok_per_tile - 1) / p.tok_per_tile;
+  p.t_max = (max_seqlen_q + 2 * p.tok_per_tile - 1) / (2 * p.tok_per_tile);
   p.n_items = static_cast<long long>(p.t_max) * n_seqs * p.n_hb;
   p.c1 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load();
