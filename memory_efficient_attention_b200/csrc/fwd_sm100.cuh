@@ -125,6 +125,90 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   }
 }
 
+// Maximum of 128 values (four independent 3-input max chains).
+__device__ __forceinline__ float row_max128(const float (&x)[128]) {
+  float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+#pragma unroll
+  for (int i = 0; i < 15; ++i) {
+    a0 = max3f(a0, x[8 + 8 * i + 0], x[8 + 8 * i + 1]);
+    a1 = max3f(a1, x[8 + 8 * i + 2], x[8 + 8 * i + 3]);
+    a2 = max3f(a2, x[8 + 8 * i + 4], x[8 + 8 * i + 5]);
+    a3 = max3f(a3, x[8 + 8 * i + 6], x[8 + 8 * i + 7]);
+  }
+  a0 = max3f(a0, x[4], x[5]);
+  a1 = max3f(a1, x[6], x[7]);
+  return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+}
+
+// Maximum over the row of c1*S(c) (+ slope2*c with ALiBi), without the per-tile constant.
+template <bool ALIBI>
+__device__ __forceinline__ float tile_score_max(const float (&x)[128], float c1, float slope2) {
+  if constexpr (!ALIBI) {
+    return row_max128(x) * c1;
+  } else {
+    const uint64_t c1x2 = f2_pack(c1, c1);
+    const uint64_t inc = f2_pack(2.f * slope2, 2.f * slope2);
+    float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+    for (int c32 = 0; c32 < 4; ++c32) {
+      uint64_t cb = f2_pack(slope2 * static_cast<float>(c32 * 32),
+                            slope2 * static_cast<float>(c32 * 32 + 1));
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int c = c32 * 32 + 2 * i;
+        float e0, e1;
+        f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), c1x2, cb), e0, e1);
+        if (i & 1)
+          m1 = max3f(m1, e0, e1);
+        else
+          m0 = max3f(m0, e0, e1);
+        cb = f2_add(cb, inc);
+      }
+    }
+    return fmaxf(m0, m1);
+  }
+}
+
+// p(c) = 2^(c1*x(c) + slope2*c - off) (slope2 term only with ALiBi) for the 128 columns of this
+// thread's row, packed to 16-bit pairs and stored over the first 64 TMEM columns at t_s.
+// Returns the row sum of p in fp32 and, in emax, the largest exponent seen.
+template <bool BF16, bool ALIBI>
+__device__ __forceinline__ float exp_tile_to_tmem(const float (&x)[128], float c1, float slope2,
+                                                  float off, uint32_t t_s, float& emax) {
+  const uint64_t c1x2 = f2_pack(c1, c1);
+  const uint64_t inc = f2_pack(2.f * slope2, 2.f * slope2);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int c4 = 0; c4 < 4; ++c4) {
+    uint64_t cb = ALIBI ? f2_pack(slope2 * static_cast<float>(c4 * 32) - off,
+                                  slope2 * static_cast<float>(c4 * 32 + 1) - off)
+                        : f2_pack(-off, -off);
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = c4 * 32 + 2 * i;
+      float e0, e1;
+      f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), c1x2, cb), e0, e1);
+      if (ALIBI) cb = f2_add(cb, inc);
+      if (i & 1)
+        m1 = max3f(m1, e0, e1);
+      else
+        m0 = max3f(m0, e0, e1);
+      const float p0 = ex2_approx(e0);
+      const float p1 = ex2_approx(e1);
+      acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+      pk[i] = pack2<BF16>(p0, p1);
+    }
+    tmem_st16(t_s + c4 * 16, pk);
+  }
+  emax = fmaxf(m0, m1);
+  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  float r0, r1;
+  f2_unpack(t, r0, r1);
+  return r0 + r1;
+}
+
 // End of a role: every thread of the CTA arrives here (from its own code path) before the
 // tcgen05 issuer warp releases tensor memory.
 __device__ __forceinline__ void fwd_teardown(bool owner, uint32_t tmem, uint32_t ncols) {
@@ -229,7 +313,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int a = 0; a < C::ATOMS; ++a)
               tma_load_3d(dst + a * C::ATOM_BYTES, w ? &tm_v : &tm_k, BAR(B_KVF + s), a * 64, g,
-                          it.k0 + j * 128);
+                          it.k0 + (nmax - 1 - j) * 128);
             ++kv_cnt;
           }
         }
@@ -275,8 +359,11 @@ __global__ void __launch_bounds__(384, 1)
           bool v_ready = false;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int nh = it.n_kv[h];
-            if (j >= 1 && j <= nh) {
+            // Tiles are visited from the last (diagonal) one down to tile 0, so the largest
+            // scores come first and the lazy O rescale rarely fires. Sub-tile h joins at
+            // iteration first_h = nmax - n_h (its own last tile).
+            const int first_h = nmax - it.n_kv[h];
+            if (j >= first_h + 1 && it.n_kv[h] > 0) {
               // ---- O_h += P_h(j-1) V_{j-1}
               if (!v_ready) {
                 ok = mbar_wait(BAR(B_KVF + vs), ((base + 2 * j - 1) / C::NS) & 1u, abort_flag,
@@ -286,7 +373,7 @@ __global__ void __launch_bounds__(384, 1)
               }
               ok = mbar_wait(BAR(B_PF + h), pv_cnt[h] & 1u, abort_flag, tmo, ecode | 3);
               if (!ok) break;
-              if (j == 1) {
+              if (j == first_h + 1) {
                 ok = mbar_wait(BAR(B_OE + h), (oe_cnt[h] & 1u) ^ 1u, abort_flag, tmo, ecode | 4);
                 if (!ok) break;
                 ++oe_cnt[h];
@@ -297,12 +384,12 @@ __global__ void __launch_bounds__(384, 1)
               for (int kk = 0; kk < C::BN / 16; ++kk) {
                 const uint64_t bd = umma_desc_sw128(vbase + kk * 2048, C::ATOM_BYTES, 1024);
                 mma_ts(tmem + C::TM_O + h * D, tmem + h * 128 + kk * 8, bd, IDESC_PV,
-                       (j == 1 && kk == 0) ? 0u : 1u);
+                       (j == first_h + 1 && kk == 0) ? 0u : 1u);
               }
               ++pv_cnt[h];
-              if (j == nh) mma_commit(BAR(B_OF + h));
+              if (j == nmax) mma_commit(BAR(B_OF + h));
             }
-            if (j < nh) {
+            if (j < nmax && j >= first_h && it.n_kv[h] > 0) {
               // ---- S_h = Q_h K_j^T
               const uint32_t kbase = kv_s0 + ks * C::TILE_BYTES;
               const uint32_t qbase = q_s + h * C::TILE_BYTES;
@@ -369,7 +456,8 @@ __global__ void __launch_bounds__(384, 1)
       float slope2 = 0.f;
       if constexpr (ALIBI) slope2 = __ldg(p.slopes + head) * LOG2E;
       float m_ref = -INFINITY, l = 0.f;
-      for (int j = 0; j < nh; ++j) {
+      for (int jj = 0; jj < nh; ++jj) {
+        const int j = nh - 1 - jj;  // key tile, visited from the diagonal downwards
         ok = mbar_wait(BAR(B_SF + h), tile & 1u, abort_flag, tmo, ecode | 8);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -391,44 +479,49 @@ __global__ void __launch_bounds__(384, 1)
         //                             constant K = slope2*(kv0 - pos), p = 2^(x - (m_ref - K))
         //   general path:             x = score,                        p = 2^(x - m_ref)
         const bool fast = (p.c1 > 0.f) && (!ALIBI || CAUSAL);
-        float m_tile, kconst = 0.f;
+        float kconst = 0.f;
+        bool resc = false;
+        float alpha = 1.f;
         if (fast) {
-          if constexpr (ALIBI) {
-            const uint64_t c1x2 = f2_pack(p.c1, p.c1);
-            const uint64_t inc = f2_pack(2.f * slope2, 2.f * slope2);
-#pragma unroll
-            for (int c32 = 0; c32 < 4; ++c32) {
-              uint64_t cb = f2_pack(slope2 * static_cast<float>(c32 * 32),
-                                    slope2 * static_cast<float>(c32 * 32 + 1));
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int c = c32 * 32 + 2 * i;
-                f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), c1x2, cb), x[c], x[c + 1]);
-                cb = f2_add(cb, inc);
-              }
-            }
-            kconst = slope2 * static_cast<float>(kv0 - pos);
-          }
+          // score(c) = c1*S(c) + slope2*c + kconst; exponent e(c) = score(c) - m_ref is formed in
+          // one packed FMA per column pair: e = c1*S + (slope2*c - off), off = m_ref - kconst.
+          if constexpr (ALIBI) kconst = slope2 * static_cast<float>(kv0 - pos);
           if (need_mask) {
 #pragma unroll
             for (int c = 0; c < 128; ++c)
               if (c > limit) x[c] = -INFINITY;
           }
-          float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
-#pragma unroll
-          for (int i = 0; i < 15; ++i) {
-            a0 = max3f(a0, x[8 + 8 * i + 0], x[8 + 8 * i + 1]);
-            a1 = max3f(a1, x[8 + 8 * i + 2], x[8 + 8 * i + 3]);
-            a2 = max3f(a2, x[8 + 8 * i + 4], x[8 + 8 * i + 5]);
-            a3 = max3f(a3, x[8 + 8 * i + 6], x[8 + 8 * i + 7]);
+          // Tiles are visited diagonal-first, so once a reference maximum exists the next tile
+          // rarely exceeds it by more than 2^8: exponentiate against it straight away and take
+          // the tile maximum on the side; redo the tile in the rare case it does.
+          const bool speculate = __all_sync(0xffffffffu, m_ref != -INFINITY);
+          if (!speculate) {
+            const float m_tile = tile_score_max<ALIBI>(x, p.c1, slope2) + kconst;
+            const float m_new = fmaxf(m_ref, m_tile);
+            resc = m_new > m_ref + 8.0f;
+            if (resc) {
+              alpha = ex2_approx(m_ref - m_new);
+              l *= alpha;
+              m_ref = m_new;
+            }
           }
-          a0 = max3f(a0, x[4], x[5]);
-          a1 = max3f(a1, x[6], x[7]);
-          const float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-          if constexpr (ALIBI)
-            m_tile = mx + kconst;
-          else
-            m_tile = mx * p.c1;
+          const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+          float emax;
+          float rs = exp_tile_to_tmem<BF16, ALIBI>(x, p.c1, slope2, m_use - kconst, t_s, emax);
+          if (speculate) {
+            const bool over = emax > 8.0f;
+            if (__any_sync(0xffffffffu, over)) {
+              if (over) {
+                const float m_tile = emax + m_use;
+                resc = true;
+                alpha = ex2_approx(m_ref - m_tile);
+                l *= alpha;
+                m_ref = m_tile;
+              }
+              rs = exp_tile_to_tmem<BF16, ALIBI>(x, p.c1, slope2, m_ref - kconst, t_s, emax);
+            }
+          }
+          l += rs;
         } else {
           const float dd0 = static_cast<float>(kv0 - pos);
 #pragma unroll
@@ -438,55 +531,21 @@ __global__ void __launch_bounds__(384, 1)
             if (need_mask && c > limit) v = -INFINITY;
             x[c] = v;
           }
-          float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
-#pragma unroll
-          for (int i = 0; i < 31; ++i) {
-            a0 = fmaxf(a0, x[4 + 4 * i + 0]);
-            a1 = fmaxf(a1, x[4 + 4 * i + 1]);
-            a2 = fmaxf(a2, x[4 + 4 * i + 2]);
-            a3 = fmaxf(a3, x[4 + 4 * i + 3]);
+          const float m_tile = row_max128(x);
+          const float m_new = fmaxf(m_ref, m_tile);
+          resc = m_new > m_ref + 8.0f;
+          if (resc) {
+            alpha = ex2_approx(m_ref - m_new);
+            l *= alpha;
+            m_ref = m_new;
           }
-          m_tile = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+          const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+          float unused;
+          l += exp_tile_to_tmem<BF16, false>(x, 1.f, 0.f, m_use, t_s, unused);
         }
-        const float m_new = fmaxf(m_ref, m_tile);
-        const bool resc = m_new > m_ref + 8.0f;
-        float alpha = 1.f;
-        if (resc) {
-          alpha = ex2_approx(m_ref - m_new);
-          l *= alpha;
-          m_ref = m_new;
-        }
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // p = 2^(mul*x - off) on pairs, summed in four independent pair accumulators
-        const float mul = (fast && !ALIBI) ? p.c1 : 1.f;
-        const float off = m_use - kconst;
-        const uint64_t mulx2 = f2_pack(mul, mul);
-        const uint64_t negoff = f2_pack(-off, -off);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint64_t e =
-                f2_fma(f2_pack(x[c4 * 32 + 2 * i], x[c4 * 32 + 2 * i + 1]), mulx2, negoff);
-            float e0, e1;
-            f2_unpack(e, e0, e1);
-            const float p0 = ex2_approx(e0);
-            const float p1 = ex2_approx(e1);
-            acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-            pk[i] = pack2<BF16>(p0, p1);
-          }
-          tmem_st16(t_s + c4 * 16, pk);
-        }
-        {
-          const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-          float r0, r1;
-          f2_unpack(t, r0, r1);
-          l += r0 + r1;
-        }
-        // O_h holds tiles < j and its last PV has completed (it was issued before QK_h(j)).
-        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        // O_h holds the tiles visited before this one and its last PV has completed (it was
+        // issued before this QK).
+        if (jj > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
           for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t o[32];
