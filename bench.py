@@ -168,22 +168,36 @@ def dist_setup(args):
     return world, rank, local
 
 
+def _collective_device():
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def dist_max(x: float, world: int) -> float:
+    """The maximum of x over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_collective_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
 def barrier(world):
+    """All ranks meet, then this rank's device is drained."""
     import torch
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def aggregate_throughput(units_per_rank: float, world: int, ms_max_over_ranks: float) -> float:
+    """Whole-job throughput of independent replicas: the units all ranks processed divided by
+    the slowest rank's time (units per second)."""
+    return world * units_per_rank / (ms_max_over_ranks * 1e-3)
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -402,10 +416,11 @@ def run_ours(args, world, rank, local):
         e2e = {"h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e}
         if do_fwd:
-            e2e.update({"value": world * flops / (e2e_fwd_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            e2e.update({"value": aggregate_throughput(flops, world, e2e_fwd_ms) / 1e12,
+                        "unit": "TFLOP/s",
                         "fwd_ms": e2e_fwd_ms})
         if do_dec:
-            e2e.update({"decode_value": world * dbytes / (e2e_dec_ms * 1e-3) / 1e9,
+            e2e.update({"decode_value": aggregate_throughput(dbytes, world, e2e_dec_ms) / 1e9,
                         "decode_unit": "GB/s", "decode_ms": e2e_dec_ms})
             if not do_fwd:
                 e2e.update({"value": e2e["decode_value"], "unit": "GB/s"})
@@ -427,7 +442,8 @@ def run_ours(args, world, rank, local):
     line["config"] = cfg
     if do_fwd:
         fwd_tf = flops / (fwd_ms * 1e-3) / 1e12
-        line.update({"value": world * fwd_tf, "unit": "TFLOP/s"})
+        line.update({"value": aggregate_throughput(flops, world, fwd_ms) / 1e12,
+                     "unit": "TFLOP/s"})
         peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         line["roofline"] = {"bound": "tensor", "achieved": fwd_tf, "peak": peak,
                             "unit": "TFLOP/s", "frac": fwd_tf / peak,
@@ -438,7 +454,8 @@ def run_ours(args, world, rank, local):
     if do_dec:
         gbs = dbytes / (dec_ms * 1e-3) / 1e9
         hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        dec_obj = {"metric": "decode KV GB/s", "value": world * gbs, "unit": "GB/s",
+        dec_obj = {"metric": "decode KV GB/s",
+                   "value": aggregate_throughput(dbytes, world, dec_ms) / 1e9, "unit": "GB/s",
                    "ms_per_call": dec_ms,
                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                                 "frac": gbs / hbm,
@@ -448,7 +465,8 @@ def run_ours(args, world, rank, local):
                                 "bytes_per_call": dbytes}}
         line["decode"] = dec_obj
         if not do_fwd:
-            line.update({"value": world * gbs, "unit": "GB/s", "roofline": dec_obj["roofline"]})
+            line.update({"value": dec_obj["value"], "unit": "GB/s",
+                         "roofline": dec_obj["roofline"]})
     line["clocks"] = clk
     line["gpu_launches"] = launches_per_step * args.steps
     if e2e is not None:

@@ -172,6 +172,20 @@ int mea_device_error(int* code, int clear);
  */
 void mea_set_wait_timeout_ns(unsigned long long ns);
 
+/*
+ * mea_wait_selftest — exercises the bounded wait that every kernel uses, with nothing else in
+ * flight: one warp initialises a shared-memory mbarrier (arrival count 1) and waits on its
+ * first phase with the given bound (`timeout_ns`, 0 means the current mea_set_wait_timeout_ns
+ * value). With `arrive` != 0 the warp first arrives itself, so the wait completes at once and
+ * the error word stays 0; with `arrive` == 0 nothing ever arrives, the wait gives up after the
+ * bound, records MEA_SELFTEST_WAIT_CODE in the device error word (if it was 0) and the kernel
+ * returns normally. This is how a caller (or a test) checks that a timed-out wait leaves the
+ * context usable and reports through mea_device_error. Asynchronous on `stream`; returns
+ * MEA_OK, or MEA_ERR_CUDA if the launch fails.
+ */
+#define MEA_SELFTEST_WAIT_CODE 0x7f01
+int mea_wait_selftest(unsigned long long timeout_ns, int arrive, void* stream);
+
 /* mea_version — library version string. */
 const char* mea_version(void);
 

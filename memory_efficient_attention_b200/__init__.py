@@ -270,3 +270,12 @@ def device_error(clear: bool = True) -> int:
 
 def set_wait_timeout_ns(ns: int) -> None:
     _lib.load().mea_set_wait_timeout_ns(int(ns))
+
+
+def wait_selftest(timeout_ns: int, arrive: bool, device=None) -> None:
+    """Runs the library's bounded wait on a barrier that is (arrive=True) or is never
+    (arrive=False) completed; in the second case the device error word afterwards holds
+    MEA_SELFTEST_WAIT_CODE. Asynchronous on the device's current stream."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _lib.check(_lib.load().mea_wait_selftest(int(timeout_ns), 1 if arrive else 0, _stream(dev)),
+               "mea_wait_selftest")

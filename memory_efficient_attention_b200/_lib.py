@@ -27,10 +27,11 @@ MEA_F16 = 0
 MEA_BF16 = 1
 MEA_MASK_NONE = 0
 MEA_MASK_CAUSAL = 1
+MEA_SELFTEST_WAIT_CODE = 0x7F01
 
 EXPORTS = ("mea_forward", "mea_decode_workspace_size", "mea_decode_splitkv",
            "mea_decode_splitkv_noalloc", "mea_status_string", "mea_device_error",
-           "mea_set_wait_timeout_ns", "mea_version")
+           "mea_set_wait_timeout_ns", "mea_wait_selftest", "mea_version")
 
 _lib = None
 
@@ -62,6 +63,8 @@ def load() -> ctypes.CDLL:
     lib.mea_device_error.restype = ci
     lib.mea_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
     lib.mea_set_wait_timeout_ns.restype = None
+    lib.mea_wait_selftest.argtypes = [ctypes.c_ulonglong, ci, vp]
+    lib.mea_wait_selftest.restype = ci
     lib.mea_version.argtypes = []
     lib.mea_version.restype = ctypes.c_char_p
     _lib = lib

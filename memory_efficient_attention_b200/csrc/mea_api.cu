@@ -217,6 +217,26 @@ int noalloc_scratch_address(void** ptr) {
 
 }  // namespace
 
+namespace mea {
+// One warp; lane 0 owns the barrier. The wait is the same bounded mbar_wait the kernels use.
+__global__ void mea_wait_selftest_kernel(unsigned long long timeout_ns, int arrive) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(b, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    if (arrive) mbar_arrive(b);
+    mbar_wait(b, 0, &abort_flag, timeout_ns, MEA_SELFTEST_WAIT_CODE);
+  }
+  __syncwarp();
+}
+}  // namespace mea
+
 extern "C" {
 
 const char* mea_version(void) { return "mea 0.1.0 (sm_100a)"; }
@@ -257,6 +277,13 @@ int mea_device_error(int* code, int clear) {
     if (cudaMemcpyToSymbol(mea::g_mea_error, &z, sizeof(z)) != cudaSuccess) return MEA_ERR_CUDA;
   }
   return MEA_OK;
+}
+
+
+int mea_wait_selftest(unsigned long long timeout_ns, int arrive, void* stream) {
+  const unsigned long long t = timeout_ns ? timeout_ns : g_timeout_ns.load();
+  mea::mea_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(t, arrive);
+  return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
 
 int mea_forward(const void* q, const void* k, const void* v, void* out, float* lse,
