@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(384, 1)
                 if (!ok) break;
                 v_ready = true;
               }
-              ok = mbar_wait(BAR(B_PF + h), pv_cnt[h] & 1u, abort_flag, tmo, ecode | 3);
+              ok = mbar_wait_spin(BAR(B_PF + h), pv_cnt[h] & 1u, abort_flag, tmo, ecode | 3);
               if (!ok) break;
               if (j == first_h + 1) {
                 ok = mbar_wait(BAR(B_OE + h), (oe_cnt[h] & 1u) ^ 1u, abort_flag, tmo, ecode | 4);

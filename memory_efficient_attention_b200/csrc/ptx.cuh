@@ -77,6 +77,46 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Non-blocking probe of a phase (cheaper than try_wait when the phase has already completed).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait with a non-blocking probe first: the tcgen05 issuer mostly waits on phases that
+// completed long ago, and every cycle it spends there leaves the tensor pipe without work.
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               uint64_t timeout_ns, unsigned code) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait(bar, parity, abort, timeout_ns, code);
+}
+
+// Bounded wait that polls with test_wait instead of suspending in try_wait: for a thread with
+// nothing else to do whose wake-up latency is on the critical path (the tcgen05 issuer).
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               uint64_t timeout_ns, unsigned code) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > timeout_ns) {
+      atomicCAS(&g_mea_error, 0u, code);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library).
 // ------------------------------------------------------------------------------------------
