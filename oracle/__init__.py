@@ -10,6 +10,7 @@ Parity unpinned (beyond limits and symmetry checks): the non-causal ALiBi form
 from .core import (  # noqa: F401
     alibi_slopes,
     attention,
+    attention_backward,
     attention_bruteforce,
     attention_probs,
     attention_rows,

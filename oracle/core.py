@@ -35,7 +35,10 @@ Readings where the pages are silent (each is listed in the design doc):
   beyond its limits);
 * lse is the natural log of the row's sum of exp(scaled, biased scores); a row with no
   admissible key has out = 0 and lse = -inf;
-* the split-KV merge combines chunk results by their log-sum-exp (plain algebra of the softmax).
+* the split-KV merge combines chunk results by their log-sum-exp (plain algebra of the softmax);
+* the backward pass is the derivative of the forward definition with respect to q, k and v for a
+  given output gradient (the pages time the forward and the backward of this attention,
+  [yifor 五大] "效能對比", but print no formula); the ALiBi slopes and the masks are constants.
 
 Everything is computed in float64 from the exact upcast of the fp16/bf16 inputs. The softmax is
 the two-pass, max-subtracted textbook form over the whole row: there is no tiling and no online
@@ -58,6 +61,7 @@ __all__ = [
     "lse_merge",
     "split_attention_chunks",
     "attention_bruteforce",
+    "attention_backward",
 ]
 
 F64 = torch.float64
@@ -308,3 +312,45 @@ def attention_bruteforce(q, k, v, seqlens_q: Sequence[int], seqlens_k: Sequence[
                     acc += w[u] * vf[u][g][e]
                 out[t][h][e] = acc / z
     return out, lse
+
+
+def attention_backward(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool,
+                       slopes: Optional[torch.Tensor] = None):
+    """Gradients ``(dq, dk, dv)`` of ``L = sum(out * dout)`` for the :func:`attention` definition,
+    in float64, with the shapes of q, k and v.
+
+    The definition differentiated by hand, per segment and query head h (key/value head
+    g = h // R), with ``P = softmax(S)`` the row softmax of the scaled, biased, masked scores:
+
+    * ``dV_g += P^T dO``                       (out = P V)
+    * ``dP = dO V^T``
+    * ``dS = P * (dP - rowsum(dO * out))``      (softmax Jacobian: ``rowsum(P * dP) = rowsum(dO * out)``)
+    * ``dQ = scale * dS K``,  ``dK_g += scale * dS^T Q``   (S = scale * Q K^T + bias)
+
+    The heads of a group add into the same dK_g, dV_g (the key/value head is shared, [gqa-snippets]).
+    Masked entries have P = 0 and contribute nothing; rows without an admissible key have zero
+    gradients.
+    """
+    cu_q, cu_k, r = _check(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    assert dout.shape == q.shape
+    q64, k64, v64, do64 = q.to(F64), k.to(F64), v.to(F64), dout.to(F64)
+    dq = torch.zeros_like(q64)
+    dk = torch.zeros_like(k64)
+    dv = torch.zeros_like(v64)
+    for s in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[s], cu_q[s + 1], cu_k[s], cu_k[s + 1]
+        if q1 == q0 or k1 == k0:
+            continue
+        for h in range(q.shape[1]):
+            g = h // r
+            qs, ks, vs, dos = q64[q0:q1, h], k64[k0:k1, g], v64[k0:k1, g], do64[q0:q1, h]
+            sc = _segment_scores(qs, ks, scale, causal, None if slopes is None else slopes[h])
+            pr, _ = _softmax_rows(sc)
+            out = pr @ vs
+            dv[k0:k1, g] += pr.T @ dos
+            dp = dos @ vs.T
+            delta = (dos * out).sum(dim=-1, keepdim=True)
+            ds = pr * (dp - delta)
+            dq[q0:q1, h] = scale * (ds @ ks)
+            dk[k0:k1, g] += scale * (ds.T @ qs)
+    return dq, dk, dv
