@@ -155,6 +155,39 @@ int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void
                                float scale, int mask_kind, const float* alibi_slopes, int dtype,
                                int split_keys, void* stream);
 
+/*
+ * mea_backward_workspace_size — bytes of workspace mea_backward needs: one fp32 per (query head,
+ * query token) for delta = rowsum(dout * out), plus 256 bytes of alignment slack.
+ */
+size_t mea_backward_workspace_size(int total_q, int n_heads_q);
+
+/*
+ * mea_backward — gradients of the packed attention of mea_forward (training backward).
+ *
+ * For L = sum(out * dout), computes dq = dL/dq, dk = dL/dk, dv = dL/dv of the definition above
+ * (the same segments, masks, GQA grouping, ALiBi slopes and scale as the forward call), as the
+ * derivative of the forward definition: with P the row softmax of the scaled, biased, masked
+ * scores, dS = P * (dout V^T - rowsum(dout * out)), dq = scale * dS K, dk = scale * dS^T Q
+ * (summed over the heads of a KV group), dv = P^T dout (likewise summed).
+ *   q, k, v, out  DEVICE, the forward's inputs and output (same layout and dtype as mea_forward).
+ *   lse           DEVICE fp32 [n_heads_q, total_q], the forward's lse (required).
+ *   dout          DEVICE gradient of out, layout and dtype of out.
+ *   dq, dk, dv    DEVICE outputs, layouts of q, k, v; every element is written (keys no query
+ *                 sees and rows that see no key get 0).
+ *   n_seqs        1 .. 65535 segments.
+ *   max_seqlen_q/k upper bounds on every L_q / L_k (they size the grids).
+ *   workspace     DEVICE, at least mea_backward_workspace_size(total_q, n_heads_q) bytes, owned
+ *                 by the caller; 16-byte aligned.
+ * No atomics: the result is deterministic. Asynchronous on `stream`. Returns MEA_OK or a
+ * negative mea_status (MEA_ERR_WORKSPACE when the workspace is missing or too small).
+ */
+int mea_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q,
+                 const int32_t* cu_seqlens_k, int n_seqs, int total_q, int total_k,
+                 int max_seqlen_q, int max_seqlen_k, int n_heads_q, int n_heads_kv, int head_dim,
+                 float scale, int mask_kind, const float* alibi_slopes, int dtype, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
 /* mea_status_string — a static English description of a mea_status value. */
 const char* mea_status_string(int status);
 

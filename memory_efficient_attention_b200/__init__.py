@@ -99,6 +99,49 @@ def attention_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out, lse
 
 
+def backward_workspace_size(total_q: int, n_heads_q: int) -> int:
+    return int(_lib.load().mea_backward_workspace_size(int(total_q), int(n_heads_q)))
+
+
+def attention_packed_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                              out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
+                              cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                              max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,
+                              alibi_slopes: Optional[torch.Tensor] = None,
+                              scale: Optional[float] = None,
+                              workspace: Optional[torch.Tensor] = None):
+    """Gradients ``(dq, dk, dv)`` of ``sum(out * dout)`` for :func:`attention_packed` called with
+    the same arguments; ``out`` and ``lse`` are that call's results."""
+    for t in (q, k, v, out, dout):
+        if not t.is_cuda:
+            raise MeaError(_lib.MEA_ERR_DEVICE, "tensors must live on the GPU")
+    q, k, v, out, dout = (t.contiguous() for t in (q, k, v, out, dout))
+    lse = lse.contiguous()
+    tq, hq, d = q.shape
+    tk, hkv, _ = k.shape
+    if dout.shape != q.shape or out.shape != q.shape or lse.shape != (hq, tq) \
+            or lse.dtype != torch.float32 or dout.dtype != q.dtype or out.dtype != q.dtype:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "out/dout must match q; lse must be fp32 [Hq, T_q]")
+    n_seqs = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if alibi_slopes is not None:
+        alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
+    need = backward_workspace_size(tq, hq)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = _lib.load().mea_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), n_seqs, tq, tk, int(max_seqlen_q),
+        int(max_seqlen_k), hq, hkv, d, float(scale),
+        _lib.MEA_MASK_CAUSAL if causal else _lib.MEA_MASK_NONE, _ptr(alibi_slopes),
+        _dtype_code(q.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(q.device))
+    _lib.check(rc, "mea_backward")
+    return dq, dk, dv
+
+
 def decode_workspace_size(n_seqs: int, total_k: int, n_heads_q: int, n_heads_kv: int,
                           head_dim: int, split_keys: int = 0) -> int:
     return int(_lib.load().mea_decode_workspace_size(n_seqs, total_k, n_heads_q, n_heads_kv,

@@ -29,7 +29,8 @@ MEA_MASK_NONE = 0
 MEA_MASK_CAUSAL = 1
 MEA_SELFTEST_WAIT_CODE = 0x7F01
 
-EXPORTS = ("mea_forward", "mea_decode_workspace_size", "mea_decode_splitkv",
+EXPORTS = ("mea_forward", "mea_backward_workspace_size", "mea_backward",
+           "mea_decode_workspace_size", "mea_decode_splitkv",
            "mea_decode_splitkv_noalloc", "mea_status_string", "mea_device_error",
            "mea_set_wait_timeout_ns", "mea_wait_selftest", "mea_version")
 
@@ -49,6 +50,11 @@ def load() -> ctypes.CDLL:
     lib.mea_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci,
                                 vp, ci, vp]
     lib.mea_forward.restype = ci
+    lib.mea_backward_workspace_size.argtypes = [ci, ci]
+    lib.mea_backward_workspace_size.restype = sz
+    lib.mea_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
+                                 ci, ci, ci, cf, ci, vp, ci, vp, sz, vp]
+    lib.mea_backward.restype = ci
     lib.mea_decode_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci]
     lib.mea_decode_workspace_size.restype = sz
     lib.mea_decode_splitkv.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp,

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/mea.h"
+#include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "ptx.cuh"
@@ -113,6 +114,48 @@ int launch_fwd_d(bool causal, bool alibi, const CUtensorMap& tq, const CUtensorM
                  : launch_fwd_t<D, BF16, true, false>(tq, tk, tv, p, grid, s);
   return alibi ? launch_fwd_t<D, BF16, false, true>(tq, tk, tv, p, grid, s)
                : launch_fwd_t<D, BF16, false, false>(tq, tk, tv, p, grid, s);
+}
+
+// ------------------------------------------------------------------------------------------
+// Backward launch dispatch.
+// ------------------------------------------------------------------------------------------
+template <typename K>
+bool set_smem_once(K kern, uint32_t smem, std::once_flag (&once)[kMaxDevices]) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t err = cudaSuccess;
+  std::call_once(once[dev], [&] {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  return err == cudaSuccess;
+}
+
+template <int D, bool BF16, bool CAUSAL, bool ALIBI>
+int launch_bwd_t(const mea::BwdParams& p, int max_q, int max_k, cudaStream_t stream) {
+  constexpr uint32_t smem = mea::BwdCfg<D>::SMEM;
+  auto kdkdv = mea::mea_bwd_dkdv_kernel<D, BF16, CAUSAL, ALIBI>;
+  auto kdq = mea::mea_bwd_dq_kernel<D, BF16, CAUSAL, ALIBI>;
+  static std::once_flag once_a[kMaxDevices], once_b[kMaxDevices];
+  if (!set_smem_once(kdkdv, smem, once_a) || !set_smem_once(kdq, smem, once_b))
+    return MEA_ERR_CUDA;
+  const long long rows = static_cast<long long>(p.total_q) * p.hq;
+  if (rows > 0)
+    mea::mea_bwd_pre_kernel<D, BF16><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(p);
+  if (max_k > 0)
+    kdkdv<<<dim3((max_k + 63) / 64, p.n_seqs, p.hkv), 128, smem, stream>>>(p);
+  if (max_q > 0)
+    kdq<<<dim3((max_q + 63) / 64, p.n_seqs, p.hq), 128, smem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+int launch_bwd_d(bool causal, bool alibi, const mea::BwdParams& p, int mq, int mk,
+                 cudaStream_t s) {
+  if (causal)
+    return alibi ? launch_bwd_t<D, BF16, true, true>(p, mq, mk, s)
+                 : launch_bwd_t<D, BF16, true, false>(p, mq, mk, s);
+  return alibi ? launch_bwd_t<D, BF16, false, true>(p, mq, mk, s)
+               : launch_bwd_t<D, BF16, false, false>(p, mq, mk, s);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -284,6 +327,74 @@ int mea_wait_selftest(unsigned long long timeout_ns, int arrive, void* stream) {
   const unsigned long long t = timeout_ns ? timeout_ns : g_timeout_ns.load();
   mea::mea_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(t, arrive);
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+size_t mea_backward_workspace_size(int total_q, int n_heads_q) {
+  if (total_q < 0 || n_heads_q < 1) return 0;
+  return static_cast<size_t>(total_q) * static_cast<size_t>(n_heads_q) * sizeof(float) + 256;
+}
+
+int mea_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q,
+                 const int32_t* cu_seqlens_k, int n_seqs, int total_q, int total_k,
+                 int max_seqlen_q, int max_seqlen_k, int n_heads_q, int n_heads_kv, int head_dim,
+                 float scale, int mask_kind, const float* alibi_slopes, int dtype, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !cu_seqlens_q ||
+      !cu_seqlens_k)
+    return MEA_ERR_NULL;
+  if (n_seqs < 1 || n_seqs > 65535 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 ||
+      max_seqlen_k < 0 || max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return MEA_ERR_SHAPE;
+  if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
+  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
+  if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
+  if (!std::isfinite(scale)) return MEA_ERR_SCALE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
+      (alibi_slopes && !aligned(alibi_slopes, 4)))
+    return MEA_ERR_ALIGN;
+  if (!workspace || !aligned(workspace, 16) ||
+      workspace_bytes < mea_backward_workspace_size(total_q, n_heads_q))
+    return MEA_ERR_WORKSPACE;
+  DeviceInfo di;
+  if (int rc = current_device_info(di); rc != MEA_OK) return rc;
+  if (total_q == 0 && total_k == 0) return MEA_OK;
+
+  mea::BwdParams p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.out = out;
+  p.lse = lse;
+  p.dout = dout;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.delta = static_cast<float*>(workspace);
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.slopes = alibi_slopes;
+  p.n_seqs = n_seqs;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.hq = n_heads_q;
+  p.hkv = n_heads_kv;
+  p.R = n_heads_q / n_heads_kv;
+  p.scale = scale;
+  p.c1 = scale * 1.4426950408889634f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool causal = mask_kind == MEA_MASK_CAUSAL;
+  const bool alibi = alibi_slopes != nullptr;
+  if (head_dim == 128)
+    return dtype == MEA_BF16
+               ? launch_bwd_d<128, true>(causal, alibi, p, max_seqlen_q, max_seqlen_k, s)
+               : launch_bwd_d<128, false>(causal, alibi, p, max_seqlen_q, max_seqlen_k, s);
+  return dtype == MEA_BF16
+             ? launch_bwd_d<64, true>(causal, alibi, p, max_seqlen_q, max_seqlen_k, s)
+             : launch_bwd_d<64, false>(causal, alibi, p, max_seqlen_q, max_seqlen_k, s);
 }
 
 int mea_forward(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -125,6 +125,50 @@ def test_decode_workspace_size(lib):
     assert dec(lib, ws=A + 16, split=64) == _lib.MEA_ERR_WORKSPACE
 
 
+def bwd(lib, **kw):
+    args = dict(q=A, k=A, v=A, out=A, lse=A, dout=A, dq=A, dk=A, dv=A, cu_q=A, cu_k=A, n_seqs=2,
+                total_q=100, total_k=120, max_q=60, max_k=70, hq=8, hkv=2, d=128, scale=0.1,
+                mask=1, slopes=None, dtype=1, ws=A, ws_bytes=1 << 20, stream=None)
+    args.update(kw)
+    return lib.mea_backward(args["q"], args["k"], args["v"], args["out"], args["lse"],
+                            args["dout"], args["dq"], args["dk"], args["dv"], args["cu_q"],
+                            args["cu_k"], args["n_seqs"], args["total_q"], args["total_k"],
+                            args["max_q"], args["max_k"], args["hq"], args["hkv"], args["d"],
+                            args["scale"], args["mask"], args["slopes"], args["dtype"],
+                            args["ws"], args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,rc", [
+    (dict(dout=None), _lib.MEA_ERR_NULL),
+    (dict(lse=None), _lib.MEA_ERR_NULL),
+    (dict(dk=None), _lib.MEA_ERR_NULL),
+    (dict(n_seqs=0), _lib.MEA_ERR_SHAPE),
+    (dict(n_seqs=70000), _lib.MEA_ERR_SHAPE),
+    (dict(max_q=101), _lib.MEA_ERR_SHAPE),
+    (dict(max_k=121), _lib.MEA_ERR_SHAPE),
+    (dict(hq=6, hkv=4), _lib.MEA_ERR_HEADS),
+    (dict(d=96), _lib.MEA_ERR_HEAD_DIM),
+    (dict(dtype=5), _lib.MEA_ERR_DTYPE),
+    (dict(mask=-1), _lib.MEA_ERR_MASK),
+    (dict(scale=float("nan")), _lib.MEA_ERR_SCALE),
+    (dict(dq=A + 8), _lib.MEA_ERR_ALIGN),
+    (dict(dout=A + 2), _lib.MEA_ERR_ALIGN),
+    (dict(lse=A + 2), _lib.MEA_ERR_ALIGN),
+    (dict(ws=None), _lib.MEA_ERR_WORKSPACE),
+    (dict(ws=A + 4), _lib.MEA_ERR_WORKSPACE),
+    (dict(ws_bytes=100 * 8 * 4 + 255), _lib.MEA_ERR_WORKSPACE),
+])
+def test_backward_rejects(lib, kw, rc):
+    assert bwd(lib, **kw) == rc
+
+
+def test_backward_workspace_size(lib):
+    assert lib.mea_backward_workspace_size(100, 8) == 100 * 8 * 4 + 256
+    assert lib.mea_backward_workspace_size(0, 8) == 256
+    assert lib.mea_backward_workspace_size(-1, 8) == 0
+    assert lib.mea_backward_workspace_size(10, 0) == 0
+
+
 def test_python_binding_fails_loudly_without_gpu():
     import torch
     import memory_efficient_attention_b200 as mea
