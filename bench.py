@@ -39,7 +39,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--part", default="all", choices=["all", "fwd", "decode"])
+    ap.add_argument("--part", default="all", choices=["all", "fwd", "decode", "bwd"],
+                    help="all = the timed step (forward + decode) plus the backward measured "
+                         "on its own; bwd = the backward alone")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -273,11 +275,12 @@ def run_ours(args, world, rank, local):
     pk, peak_src = peaks()
     do_fwd = args.part in ("all", "fwd")
     do_dec = args.part in ("all", "decode")
+    do_bwd = args.part in ("all", "bwd")
 
     w2, w4 = workload(2), workload(4)
     g = torch.Generator(device=dev)
     # ---- forward inputs (packed causal GQA + ALiBi)
-    if do_fwd:
+    if do_fwd or do_bwd:
         g.manual_seed(w2.seed)
         tq = w2.total_q
         q = torch.randn((tq, 32, 128), generator=g, device=dev, dtype=torch.float32).bfloat16()
@@ -357,7 +360,7 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through the public API with host buffers (pinned), copies inside
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and (do_fwd or do_dec):
         h2d = d2h = 0
         e2e_fwd_ms = e2e_dec_ms = 0.0
         n_e2e = max(1, args.e2e_steps)
@@ -425,6 +428,47 @@ def run_ours(args, world, rank, local):
             if not do_fwd:
                 e2e.update({"value": e2e["decode_value"], "unit": "GB/s"})
 
+    # ---- backward on the packed prefill workload, timed on its own (not part of the step)
+    bwd_obj = None
+    if do_bwd:
+        g.manual_seed(w2.seed + 1)
+        gout = torch.randn((tq, 32, 128), generator=g, device=dev, dtype=torch.float32).bfloat16()
+        gdq, gdk, gdv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = torch.empty(mea.backward_workspace_size(tq, 32), dtype=torch.uint8, device=dev)
+        fwd_b = mea.attention_packed(q, k, v, cu, cu, max_q, causal=True, alibi_slopes=slopes,
+                                     scale=w2.scale)
+
+        def bwd():
+            mea.attention_packed_backward(q, k, v, fwd_b[0], fwd_b[1], gout, cu, cu, max_q, max_q,
+                                          causal=True, alibi_slopes=slopes, scale=w2.scale,
+                                          workspace=bws, dq=gdq, dk=gdk, dv=gdv)
+        for _ in range(args.warmup):
+            bwd()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            bwd()
+        b.record(stream)
+        barrier(world)
+        bwd_ms = dist_max(a.elapsed_time(b), world) / args.steps
+        code = mea.device_error()
+        if code:
+            raise RuntimeError(f"device error word {code:#x} during the backward")
+        bflops = 2.5 * fwd_flops(w2.seqlens_q, 32, 128)
+        btf = bflops / (bwd_ms * 1e-3) / 1e12
+        peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        bwd_obj = {"metric": "attention bwd TFLOP/s (packed causal GQA+ALiBi)",
+                   "value": aggregate_throughput(bflops, world, bwd_ms) / 1e12,
+                   "unit": "TFLOP/s", "ms_per_call": bwd_ms, "flops_per_call": bflops,
+                   "launches_per_call": 3,
+                   "roofline": {"bound": "tensor", "achieved": btf, "peak": peak,
+                                "unit": "TFLOP/s", "frac": btf / peak,
+                                "traffic": traffic_for("mea_bwd_dkdv_kernel"),
+                                "peak_kind": f"dense bf16 burst, {peak_src}",
+                                "kernel": "mea_bwd_pre_kernel + mea_bwd_dkdv_kernel + "
+                                          "mea_bwd_dq_kernel"}}
+
     if rank != 0:
         return 0
 
@@ -467,6 +511,12 @@ def run_ours(args, world, rank, local):
         if not do_fwd:
             line.update({"value": dec_obj["value"], "unit": "GB/s",
                          "roofline": dec_obj["roofline"]})
+    if bwd_obj is not None:
+        line["backward"] = bwd_obj
+        if not do_fwd and not do_dec:
+            line.update({"value": bwd_obj["value"], "unit": "TFLOP/s",
+                         "roofline": bwd_obj["roofline"], "ms_per_step": bwd_obj["ms_per_call"]})
+            line["metric"] = bwd_obj["metric"]
     line["clocks"] = clk
     line["gpu_launches"] = launches_per_step * args.steps
     if e2e is not None:

@@ -109,9 +109,12 @@ def attention_packed_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                               max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,
                               alibi_slopes: Optional[torch.Tensor] = None,
                               scale: Optional[float] = None,
-                              workspace: Optional[torch.Tensor] = None):
+                              workspace: Optional[torch.Tensor] = None,
+                              dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                              dv: Optional[torch.Tensor] = None):
     """Gradients ``(dq, dk, dv)`` of ``sum(out * dout)`` for :func:`attention_packed` called with
-    the same arguments; ``out`` and ``lse`` are that call's results."""
+    the same arguments; ``out`` and ``lse`` are that call's results. ``dq``/``dk``/``dv`` may be
+    given as preallocated contiguous outputs."""
     for t in (q, k, v, out, dout):
         if not t.is_cuda:
             raise MeaError(_lib.MEA_ERR_DEVICE, "tensors must live on the GPU")
@@ -130,7 +133,9 @@ def attention_packed_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     need = backward_workspace_size(tq, hq)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
     rc = _lib.load().mea_backward(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
         _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), n_seqs, tq, tk, int(max_seqlen_q),
