@@ -43,6 +43,10 @@ def parse():
                     help="all = the timed step (forward + decode) plus the backward measured "
                          "on its own; bwd = the backward alone")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-paged", dest="paged", action="store_false",
+                    help="skip the paged-cache decode measurement")
+    ap.add_argument("--paged-block-size", type=int, default=16,
+                    help="slots per cache block of the paged decode measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--decode-requests", type=int, default=64,
@@ -322,6 +326,36 @@ def run_ours(args, world, rank, local):
             mea.decode_splitkv(dq, dk, dv, dcu, max_k, scale=w4.scale, workspace=ws, out=dout,
                                lse=dlse)
 
+        # The same keys/values in a paged cache of 16-slot blocks (blocks in a shuffled order).
+        pbs = args.paged_block_size
+        nblk = [-(-x // pbs) for x in lk]
+        pperm = torch.randperm(sum(nblk), generator=g, device=dev).to(torch.int32)
+        ptable = torch.zeros((n_req, max(nblk)), dtype=torch.int32, device=dev)
+        pkc = torch.zeros((sum(nblk), pbs, 8, 128), dtype=torch.bfloat16, device=dev)
+        pvc = torch.zeros_like(pkc)
+        nxt, off = 0, 0
+        for b, length in enumerate(lk):
+            ids = pperm[nxt:nxt + nblk[b]]
+            ptable[b, :nblk[b]] = ids
+            full = length // pbs
+            if full:
+                pkc[ids[:full].long()] = dk[off:off + full * pbs].view(full, pbs, 8, 128)
+                pvc[ids[:full].long()] = dv[off:off + full * pbs].view(full, pbs, 8, 128)
+            rem = length - full * pbs
+            if rem:
+                pkc[int(ids[full]), :rem] = dk[off + full * pbs:off + length]
+                pvc[int(ids[full]), :rem] = dv[off + full * pbs:off + length]
+            nxt += nblk[b]
+            off += length
+        pws = torch.empty(mea.decode_workspace_size(n_req, sum(nblk) * pbs, 64, 8, 128, 0),
+                          dtype=torch.uint8, device=dev)
+        pout = torch.empty_like(dq)
+        plse = torch.empty_like(dlse)
+
+        def dec_paged():
+            mea.decode_paged(dq, pkc, pvc, ptable, dcu, max_k, scale=w4.scale, workspace=pws,
+                             out=pout, lse=plse)
+
     launches_per_step = (1 if do_fwd else 0) + (2 if do_dec else 0)
     for _ in range(args.warmup):
         if do_fwd:
@@ -428,6 +462,34 @@ def run_ours(args, world, rank, local):
             if not do_fwd:
                 e2e.update({"value": e2e["decode_value"], "unit": "GB/s"})
 
+    # ---- paged-cache decode of the same requests, timed on its own (not part of the step)
+    paged_obj = None
+    if do_dec and args.paged:
+        for _ in range(args.warmup):
+            dec_paged()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            dec_paged()
+        b.record(stream)
+        barrier(world)
+        pms = dist_max(a.elapsed_time(b), world) / args.steps
+        code = mea.device_error()
+        if code:
+            raise RuntimeError(f"device error word {code:#x} during the paged decode")
+        pgbs = dbytes / (pms * 1e-3) / 1e9
+        hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        paged_obj = {"metric": f"paged decode KV GB/s ({pbs}-slot blocks, shuffled)",
+                     "value": aggregate_throughput(dbytes, world, pms) / 1e9, "unit": "GB/s",
+                     "ms_per_call": pms, "block_size": pbs,
+                     "roofline": {"bound": "hbm", "achieved": pgbs, "peak": hbm, "unit": "GB/s",
+                                  "frac": pgbs / hbm, "traffic": None,
+                                  "peak_kind": f"HBM copy bandwidth, {peak_src}",
+                                  "kernel": "mea_decode_split_kernel<paged> + "
+                                            "mea_lse_merge_kernel",
+                                  "bytes_per_call": dbytes}}
+
     # ---- backward on the packed prefill workload, timed on its own (not part of the step)
     bwd_obj = None
     if do_bwd:
@@ -511,6 +573,8 @@ def run_ours(args, world, rank, local):
         if not do_fwd:
             line.update({"value": dec_obj["value"], "unit": "GB/s",
                          "roofline": dec_obj["roofline"]})
+    if paged_obj is not None:
+        line["paged_decode"] = paged_obj
     if bwd_obj is not None:
         line["backward"] = bwd_obj
         if not do_fwd and not do_dec:

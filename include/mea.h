@@ -188,6 +188,28 @@ int mea_backward(const void* q, const void* k, const void* v, const void* out, c
                  float scale, int mask_kind, const float* alibi_slopes, int dtype, void* workspace,
                  size_t workspace_bytes, void* stream);
 
+/*
+ * mea_decode_paged — mea_decode_splitkv over a paged K/V cache (serving layout): request b's key
+ * t (0 <= t < L_b) lives in cache block block_table[b * max_blocks + t / block_size], slot
+ * t % block_size. Same arithmetic, masks, output and workspace as mea_decode_splitkv.
+ *   k_cache, v_cache  DEVICE [num_blocks, block_size, n_heads_kv, head_dim], dtype of q.
+ *   block_table       DEVICE int32 [n_seqs, max_blocks]; entries past ceil(L_b / block_size)
+ *                     are not read. An id outside [0, num_blocks) reads as zeros (never faults).
+ *   cu_seqlens_k      DEVICE int32 [n_seqs + 1], prefix sums of the requests' key counts L_b.
+ *   block_size        16, 32, or a multiple of 64.
+ *   total_k           an upper bound on cu_seqlens_k[n_seqs] (for example num_blocks *
+ *                     block_size); it sizes the workspace exactly as in mea_decode_splitkv:
+ *                     mea_decode_workspace_size(n_seqs, total_k, ...).
+ *   max_seqlen_k      an upper bound on every L_b, at most max_blocks * block_size.
+ * Slots of a block past the end of its sequence may hold any bits (they are never used).
+ */
+int mea_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_table, const int32_t* cu_seqlens_k, void* out,
+                     float* lse, int n_seqs, int num_blocks, int block_size, int max_blocks,
+                     int total_k, int max_seqlen_k, int n_heads_q, int n_heads_kv, int head_dim,
+                     float scale, int mask_kind, const float* alibi_slopes, int dtype,
+                     void* workspace, size_t workspace_bytes, int split_keys, void* stream);
+
 /* mea_status_string — a static English description of a mea_status value. */
 const char* mea_status_string(int status);
 

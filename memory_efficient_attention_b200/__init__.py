@@ -187,6 +187,47 @@ def decode_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
     return out, lse
 
 
+def decode_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                 block_table: torch.Tensor, cu_seqlens_k: torch.Tensor, max_seqlen_k: int,
+                 alibi_slopes: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                 workspace: Optional[torch.Tensor] = None, split_keys: int = 0,
+                 total_k_bound: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None):
+    """Split-KV decode over a paged cache ``[num_blocks, block_size, Hkv, D]`` with an int32
+    ``block_table [n_seqs, max_blocks]``. Returns ``(out [n_seqs, Hq, D], lse [Hq, n_seqs])``."""
+    for t in (q, k_cache, v_cache, block_table, cu_seqlens_k):
+        if not t.is_cuda:
+            raise MeaError(_lib.MEA_ERR_DEVICE, "tensors must live on the GPU")
+    q = q.contiguous()
+    k_cache, v_cache = k_cache.contiguous(), v_cache.contiguous()
+    block_table = block_table.contiguous()
+    n, hq, d = q.shape
+    nb, bs, hkv, _ = k_cache.shape
+    if v_cache.shape != k_cache.shape or block_table.dtype != torch.int32 \
+            or block_table.dim() != 2 or block_table.shape[0] != n:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "cache / block table shapes disagree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    total = int(total_k_bound) if total_k_bound is not None else nb * bs
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_size(n, total, hq, hkv, d, split_keys),
+                                dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((hq, n), dtype=torch.float32, device=q.device)
+    if alibi_slopes is not None:
+        alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
+    rc = _lib.load().mea_decode_paged(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cu_seqlens_k), _ptr(out),
+        _ptr(lse), n, nb, bs, block_table.shape[1], total, int(max_seqlen_k), hq, hkv, d,
+        float(scale), _lib.MEA_MASK_CAUSAL, _ptr(alibi_slopes), _dtype_code(q.dtype),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), int(split_keys),
+        _stream(q.device))
+    _lib.check(rc, "mea_decode_paged")
+    return out, lse
+
+
 def decode_splitkv_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                            cu_seqlens_k: torch.Tensor, max_seqlen_k: int, out: torch.Tensor,
                            lse: Optional[torch.Tensor] = None,

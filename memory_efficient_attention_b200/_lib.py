@@ -30,7 +30,7 @@ MEA_MASK_CAUSAL = 1
 MEA_SELFTEST_WAIT_CODE = 0x7F01
 
 EXPORTS = ("mea_forward", "mea_backward_workspace_size", "mea_backward",
-           "mea_decode_workspace_size", "mea_decode_splitkv",
+           "mea_decode_workspace_size", "mea_decode_splitkv", "mea_decode_paged",
            "mea_decode_splitkv_noalloc", "mea_status_string", "mea_device_error",
            "mea_set_wait_timeout_ns", "mea_wait_selftest", "mea_version")
 
@@ -60,6 +60,9 @@ def load() -> ctypes.CDLL:
     lib.mea_decode_splitkv.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp,
                                        ci, vp, sz, ci, vp]
     lib.mea_decode_splitkv.restype = ci
+    lib.mea_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ci,
+                                     ci, cf, ci, vp, ci, vp, sz, ci, vp]
+    lib.mea_decode_paged.restype = ci
     lib.mea_decode_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf,
                                                ci, vp, ci, ci, vp]
     lib.mea_decode_splitkv_noalloc.restype = ci

@@ -26,8 +26,12 @@ struct DecParams {
   const void* q;      // [n_seqs, hq, D]
   void* out;          // [n_seqs, hq, D]
   float* lse;         // [hq, n_seqs] or null
-  const int32_t* cu_k;
+  const int32_t* cu_k;         // prefix sums of the requests' key counts
   const float* slopes;
+  const int32_t* block_table;  // paged K/V only: [n_seqs, max_blocks] cache block ids
+  int block_size;              // paged: keys per cache block (16, 32 or a multiple of 64)
+  int max_blocks;              // paged: row length of block_table
+  int num_blocks;              // paged: blocks in the cache (ids outside [0, num_blocks) read 0)
   float* ws_o;        // [n_slots, hq, D]
   float* ws_lse;      // [n_slots, hq]
   int n_seqs;
@@ -107,7 +111,9 @@ __device__ __forceinline__ int dec_chunk_start(const int32_t* cu, int b, int chu
   return acc;
 }
 
-template <int D, bool BF16, bool ALIBI>
+// PAGED: K/V live in a block cache [num_blocks, block_size, Hkv, D] addressed through a per-request
+// block table (4-D TMA maps) instead of a packed [T_k, Hkv, D] tensor (3-D maps).
+template <int D, bool BF16, bool ALIBI, bool PAGED = false>
 __global__ void __launch_bounds__(160, 1)
     mea_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
@@ -162,19 +168,69 @@ __global__ void __launch_bounds__(160, 1)
       const int n_tiles = (nk + C::BK - 1) / C::BK;
       const int g = (hb * p.RB) / p.R;
       if (lane == 0) {
+        // Paged: the cache block ids of tile t+1 are loaded while tile t is being issued, so the
+        // table reads never wait in line behind the TMA issue.
+        constexpr int MAXPER = C::BK / 16;  // blocks per tile at the smallest block size
+        int ids_next[MAXPER] = {};
+        const int32_t* row = nullptr;
+        int per = 1, nblk = 0;
+        if constexpr (PAGED) {
+          row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+          per = p.block_size >= C::BK ? 1 : C::BK / p.block_size;
+          nblk = min((L + p.block_size - 1) / p.block_size, p.max_blocks);
+#pragma unroll
+          for (int i = 0; i < MAXPER; ++i) {
+            const int j = (key0 + i * p.block_size) / p.block_size;
+            ids_next[i] = (i < per && j < nblk) ? __ldg(row + j) : p.num_blocks;
+          }
+        }
         for (int t = 0; t < n_tiles; ++t) {
+          int ids[MAXPER];
+#pragma unroll
+          for (int i = 0; i < MAXPER; ++i) ids[i] = ids_next[i];
+          if constexpr (PAGED) {
+            const int kn = key0 + (t + 1) * C::BK;
+#pragma unroll
+            for (int i = 0; i < MAXPER; ++i) {
+              const int j = (kn + i * p.block_size) / p.block_size;
+              ids_next[i] = (t + 1 < n_tiles && i < per && j < nblk) ? __ldg(row + j)
+                                                                       : p.num_blocks;
+            }
+          }
           const uint32_t s = cnt % C::NS;
           const uint32_t ph = (cnt / C::NS) & 1u;
           ok = mbar_wait(DBAR(B_E + s), ph ^ 1u, abort_flag, tmo, ecode | 1);
           if (!ok) break;
           mbar_arrive_expect_tx(DBAR(B_F + s), C::STAGE_BYTES);
           const uint32_t dst = sbase + C::SMEM_RING + s * C::STAGE_BYTES;
-          const int tok = k0 + key0 + t * C::BK;
+          if constexpr (PAGED) {
+            // Tile keys [kt, kt + 64) of request b: one box per cache block (block sizes 16, 32:
+            // boxes of block_size rows at row offsets that keep the 128-B swizzle aligned) or a
+            // 64-row slice of one block (block sizes that are multiples of 64). Blocks past the
+            // request's last one use id num_blocks, which the TMA fills with zeros.
+            const int kt = key0 + t * C::BK;
+            const int bs = p.block_size;
+            const int r0 = bs >= C::BK ? kt % bs : 0;
 #pragma unroll
-          for (int a = 0; a < C::ATOMS; ++a) {
-            tma_load_3d(dst + a * C::ATOM_BYTES, &tm_k, DBAR(B_F + s), a * 64, g, tok);
-            tma_load_3d(dst + C::KT_BYTES + a * C::ATOM_BYTES, &tm_v, DBAR(B_F + s), a * 64, g,
-                        tok);
+            for (int i = 0; i < MAXPER; ++i) {
+              if (i >= per) break;
+              const uint32_t rows_off = static_cast<uint32_t>(i * bs * 128);
+#pragma unroll
+              for (int a = 0; a < C::ATOMS; ++a) {
+                tma_load_4d(dst + a * C::ATOM_BYTES + rows_off, &tm_k, DBAR(B_F + s), a * 64, g,
+                            r0, ids[i]);
+                tma_load_4d(dst + C::KT_BYTES + a * C::ATOM_BYTES + rows_off, &tm_v,
+                            DBAR(B_F + s), a * 64, g, r0, ids[i]);
+              }
+            }
+          } else {
+            const int tok = k0 + key0 + t * C::BK;
+#pragma unroll
+            for (int a = 0; a < C::ATOMS; ++a) {
+              tma_load_3d(dst + a * C::ATOM_BYTES, &tm_k, DBAR(B_F + s), a * 64, g, tok);
+              tma_load_3d(dst + C::KT_BYTES + a * C::ATOM_BYTES, &tm_v, DBAR(B_F + s), a * 64,
+                          g, tok);
+            }
           }
           ++cnt;
         }
@@ -242,6 +298,23 @@ __global__ void __launch_bounds__(160, 1)
         if (!ok) break;
         const uint32_t kst = sbase + C::SMEM_RING + s * C::STAGE_BYTES;
         const uint32_t vst = kst + C::KT_BYTES;
+        bool zeroed = false;
+        if constexpr (PAGED) {
+          // A cache block's slots past the sequence end may hold anything (0 * NaN is NaN in
+          // P V): zero this warp's V rows past the last key of a partial tile.
+          const int valid = nk - t * C::BK;
+          if (valid < C::BK) {
+            const int r_lo = max(valid, warp * 16), r_hi = warp * 16 + 16;
+            for (int i = lane; i < (r_hi > r_lo ? (r_hi - r_lo) * (D / 8) : 0); i += 32) {
+              const int rr = r_lo + i / (D / 8), ch = i % (D / 8);
+              const uint32_t addr = vst + (ch >> 3) * C::ATOM_BYTES + rr * 128 + ((ch & 7) << 4);
+              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u)
+                           : "memory");
+            }
+            zeroed = true;
+            __syncwarp();
+          }
+        }
         // ---- S^T fragment: rows = heads, cols = this warp's 16 keys (two n-tiles of 8)
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         {
@@ -333,6 +406,8 @@ __global__ void __launch_bounds__(160, 1)
             mma16816<BF16>(o[n + 1], pa, r2, r3);
           }
         }
+        // Generic-proxy writes to the slot must be ordered before the next TMA write into it.
+        if (PAGED && zeroed) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive(DBAR(B_E + s));
         ++cnt;

@@ -116,6 +116,23 @@ int launch_fwd_d(bool causal, bool alibi, const CUtensorMap& tq, const CUtensorM
                : launch_fwd_t<D, BF16, false, false>(tq, tk, tv, p, grid, s);
 }
 
+// 4-D tiled map over a paged cache [d3 blocks, d2 slots, d1 heads, d0] of 16-bit elements.
+bool encode_4d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {d0, d1, d2, d3};
+  cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  cuuint32_t box[4] = {b0, b1, b2, b3};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, dtype == MEA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------------------------------
 // Backward launch dispatch.
 // ------------------------------------------------------------------------------------------
@@ -161,10 +178,10 @@ int launch_bwd_d(bool causal, bool alibi, const mea::BwdParams& p, int mq, int m
 // ------------------------------------------------------------------------------------------
 // Decode launch dispatch.
 // ------------------------------------------------------------------------------------------
-template <int D, bool BF16, bool ALIBI>
+template <int D, bool BF16, bool ALIBI, bool PAGED>
 int launch_dec_t(const CUtensorMap& tk, const CUtensorMap& tv, const mea::DecParams& p,
                  int grid, int n_kv_heads, cudaStream_t stream) {
-  auto kern = mea::mea_decode_split_kernel<D, BF16, ALIBI>;
+  auto kern = mea::mea_decode_split_kernel<D, BF16, ALIBI, PAGED>;
   constexpr uint32_t smem = mea::DecCfg<D>::SMEM_TOTAL;
   static std::once_flag once[kMaxDevices];
   int dev = 0;
@@ -181,11 +198,11 @@ int launch_dec_t(const CUtensorMap& tk, const CUtensorMap& tv, const mea::DecPar
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool PAGED = false>
 int launch_dec_d(bool alibi, const CUtensorMap& tk, const CUtensorMap& tv,
                  const mea::DecParams& p, int grid, int hkv, cudaStream_t s) {
-  return alibi ? launch_dec_t<D, BF16, true>(tk, tv, p, grid, hkv, s)
-               : launch_dec_t<D, BF16, false>(tk, tv, p, grid, hkv, s);
+  return alibi ? launch_dec_t<D, BF16, true, PAGED>(tk, tv, p, grid, hkv, s)
+               : launch_dec_t<D, BF16, false, PAGED>(tk, tv, p, grid, hkv, s);
 }
 
 int auto_split_keys(int total_k, int n_hb, int sms) {
@@ -528,6 +545,81 @@ int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, f
                              : launch_dec_d<128, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
   return dtype == MEA_BF16 ? launch_dec_d<64, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
                            : launch_dec_d<64, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
+}
+
+int mea_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_table, const int32_t* cu_seqlens_k, void* out,
+                     float* lse, int n_seqs, int num_blocks, int block_size, int max_blocks,
+                     int total_k, int max_seqlen_k, int n_heads_q, int n_heads_kv, int head_dim,
+                     float scale, int mask_kind, const float* alibi_slopes, int dtype,
+                     void* workspace, size_t workspace_bytes, int split_keys, void* stream) {
+  if (!q || !k_cache || !v_cache || !block_table || !cu_seqlens_k || !out) return MEA_ERR_NULL;
+  if (n_seqs < 1 || num_blocks < 1 || max_blocks < 1 || total_k < 0 || max_seqlen_k < 0 ||
+      max_seqlen_k > total_k || static_cast<long long>(max_blocks) * block_size < max_seqlen_k)
+    return MEA_ERR_SHAPE;
+  if (!(block_size == 16 || block_size == 32 || (block_size >= 64 && block_size % 64 == 0)))
+    return MEA_ERR_SHAPE;
+  if (split_keys < 0 || split_keys % 64) return MEA_ERR_SHAPE;
+  if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
+  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
+  if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
+  if (!std::isfinite(scale)) return MEA_ERR_SCALE;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)) || !aligned(cu_seqlens_k, 4) || !aligned(block_table, 4) ||
+      (alibi_slopes && !aligned(alibi_slopes, 4)))
+    return MEA_ERR_ALIGN;
+  if (!workspace || !aligned(workspace, 256)) return MEA_ERR_WORKSPACE;
+  DeviceInfo di;
+  int dev_rc = MEA_OK;
+  if (split_keys == 0 && (dev_rc = current_device_info(di)) != MEA_OK) return dev_rc;
+  DecLayout L;
+  if (!dec_layout(n_seqs, total_k, n_heads_q, n_heads_kv, head_dim, split_keys,
+                  split_keys == 0 ? di.sms : 0, L))
+    return MEA_ERR_SHAPE;
+  if (workspace_bytes < L.total) return MEA_ERR_WORKSPACE;
+  if (split_keys != 0 && (dev_rc = current_device_info(di)) != MEA_OK) return dev_rc;
+
+  const int R = n_heads_q / n_heads_kv;
+  mea::DecParams p{};
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.cu_k = cu_seqlens_k;
+  p.slopes = alibi_slopes;
+  p.block_table = block_table;
+  p.block_size = block_size;
+  p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.lse_off);
+  p.n_seqs = n_seqs;
+  p.hq = n_heads_q;
+  p.R = R;
+  p.RB = decode_rb(R);
+  p.n_hb = n_heads_q / p.RB;
+  p.chunk = L.chunk;
+  p.n_slots = L.n_slots;
+  p.n_items = static_cast<long long>(L.n_slots) * p.n_hb;
+  p.c1 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+
+  CUtensorMap tk, tv;
+  const uint32_t rows = block_size < 64 ? static_cast<uint32_t>(block_size) : 64u;
+  if (!encode_4d(&tk, k_cache, dtype, head_dim, n_heads_kv, block_size, num_blocks, 64, 1, rows,
+                 1) ||
+      !encode_4d(&tv, v_cache, dtype, head_dim, n_heads_kv, block_size, num_blocks, 64, 1, rows,
+                 1))
+    return MEA_ERR_CUDA;
+  const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool alibi = alibi_slopes != nullptr;
+  if (head_dim == 128)
+    return dtype == MEA_BF16
+               ? launch_dec_d<128, true, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+               : launch_dec_d<128, false, true>(alibi, tk, tv, p, grid, n_heads_kv, s);
+  return dtype == MEA_BF16 ? launch_dec_d<64, true, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+                           : launch_dec_d<64, false, true>(alibi, tk, tv, p, grid, n_heads_kv, s);
 }
 
 int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -16,6 +16,7 @@ from .core import (  # noqa: F401
     attention_rows,
     decode,
     lse_merge,
+    paged_gather,
     segment_positions,
     split_attention_chunks,
 )

@@ -62,6 +62,7 @@ __all__ = [
     "split_attention_chunks",
     "attention_bruteforce",
     "attention_backward",
+    "paged_gather",
 ]
 
 F64 = torch.float64
@@ -354,3 +355,22 @@ def attention_backward(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, scale: float, 
             dq[q0:q1, h] = scale * (ds @ ks)
             dk[k0:k1, g] += scale * (ds.T @ qs)
     return dq, dk, dv
+
+
+def paged_gather(cache: torch.Tensor, block_table, seqlens_k: Sequence[int]) -> torch.Tensor:
+    """The packed ``[sum L_b, H, D]`` keys (or values) of a paged cache ``[num_blocks,
+    block_size, H, D]``: request b's key t is ``cache[block_table[b][t // block_size],
+    t % block_size]``.
+
+    [7minutos §4] names vLLM-style engines as the users of packed variable-length batches; their
+    K/V cache is paged through a per-request block table. The pages do not print that layout:
+    this is the plain reading (a gather), used to state paged decode as packed decode.
+    """
+    bs = cache.shape[1]
+    rows = []
+    for b, length in enumerate(seqlens_k):
+        for t in range(int(length)):
+            rows.append(cache[int(block_table[b][t // bs]), t % bs])
+    if not rows:
+        return cache.new_zeros((0,) + tuple(cache.shape[2:]))
+    return torch.stack(rows)

@@ -169,6 +169,46 @@ def test_backward_workspace_size(lib):
     assert lib.mea_backward_workspace_size(10, 0) == 0
 
 
+def paged(lib, **kw):
+    args = dict(q=A, kc=A, vc=A, table=A, cu_k=A, out=A, lse=A, n_seqs=2, num_blocks=10, bs=16,
+                max_blocks=5, total_k=160, max_k=70, hq=64, hkv=8, d=128, scale=0.1, mask=1,
+                slopes=None, dtype=1, ws=A, ws_bytes=1 << 30, split=0, stream=None)
+    args.update(kw)
+    return lib.mea_decode_paged(args["q"], args["kc"], args["vc"], args["table"], args["cu_k"],
+                                args["out"], args["lse"], args["n_seqs"], args["num_blocks"],
+                                args["bs"], args["max_blocks"], args["total_k"], args["max_k"],
+                                args["hq"], args["hkv"], args["d"], args["scale"], args["mask"],
+                                args["slopes"], args["dtype"], args["ws"], args["ws_bytes"],
+                                args["split"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,rc", [
+    (dict(table=None), _lib.MEA_ERR_NULL),
+    (dict(kc=None), _lib.MEA_ERR_NULL),
+    (dict(bs=24), _lib.MEA_ERR_SHAPE),
+    (dict(bs=8), _lib.MEA_ERR_SHAPE),
+    (dict(bs=96), _lib.MEA_ERR_SHAPE),
+    (dict(max_blocks=4), _lib.MEA_ERR_SHAPE),        # 4 x 16 < max_k = 70
+    (dict(num_blocks=0), _lib.MEA_ERR_SHAPE),
+    (dict(max_k=161), _lib.MEA_ERR_SHAPE),
+    (dict(split=100), _lib.MEA_ERR_SHAPE),
+    (dict(hq=12, hkv=8), _lib.MEA_ERR_HEADS),
+    (dict(d=80), _lib.MEA_ERR_HEAD_DIM),
+    (dict(dtype=7), _lib.MEA_ERR_DTYPE),
+    (dict(table=A + 2), _lib.MEA_ERR_ALIGN),
+    (dict(vc=A + 8), _lib.MEA_ERR_ALIGN),
+    (dict(ws=None), _lib.MEA_ERR_WORKSPACE),
+    (dict(ws=A + 16), _lib.MEA_ERR_WORKSPACE),
+])
+def test_paged_decode_rejects(lib, kw, rc):
+    assert paged(lib, **kw) == rc
+
+
+def test_paged_decode_workspace_is_the_decode_workspace(lib):
+    need = lib.mea_decode_workspace_size(2, 160, 64, 8, 128, 64)
+    assert paged(lib, ws_bytes=need - 1, split=64) == _lib.MEA_ERR_WORKSPACE
+
+
 def test_python_binding_fails_loudly_without_gpu():
     import torch
     import memory_efficient_attention_b200 as mea

@@ -410,3 +410,28 @@ def test_planted_mistakes_are_caught(kind, monkeypatch):
         except Exception:  # a crash also counts as a caught mistake
             results[pin.__name__] = False
     assert not all(results.values()), f"mutant {kind} passed every pin"
+
+
+def test_paged_gather_inverts_a_brute_force_scatter():
+    """Scatter packed keys into a shuffled block cache with explicit loops, then gather them back
+    with oracle.paged_gather: the packed tensor is recovered exactly (block sizes 16 and 64,
+    requests that end mid-block, unused blocks holding NaN)."""
+    g = torch.Generator().manual_seed(77)
+    for bs in (16, 64):
+        lens = [1, 17, 64, 100, 0, 33]
+        packed = torch.randn((sum(lens), 3, 8), generator=g, dtype=F64)
+        nblk = [-(-x // bs) for x in lens]
+        num_blocks = sum(nblk) + 3
+        perm = torch.randperm(num_blocks, generator=g).tolist()
+        cache = torch.full((num_blocks, bs, 3, 8), float("nan"), dtype=F64)
+        table = [[-1] * max(nblk) for _ in lens]
+        nxt, off = 0, 0
+        for b, length in enumerate(lens):
+            for j in range(nblk[b]):
+                table[b][j] = perm[nxt]
+                nxt += 1
+            for t in range(length):
+                cache[table[b][t // bs], t % bs] = packed[off + t]
+            off += length
+        back = oracle.paged_gather(cache, table, lens)
+        assert torch.equal(back, packed)
