@@ -517,6 +517,21 @@ def run_ours(args, world, rank, local):
         code = mea.device_error()
         if code:
             raise RuntimeError(f"device error word {code:#x} during the backward")
+        # Peak memory of one forward + backward call pair: nothing is allocated by the library.
+        torch.cuda.synchronize()
+        free0, _ = torch.cuda.mem_get_info(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        alloc0 = torch.cuda.memory_allocated(dev)
+        mea.attention_packed(q, k, v, cu, cu, max_q, causal=True, alibi_slopes=slopes,
+                             scale=w2.scale, out=fwd_b[0], lse=fwd_b[1])
+        bwd()
+        torch.cuda.synchronize()
+        free1, _ = torch.cuda.mem_get_info(dev)
+        mem_obj = {"device_bytes_allocated_by_calls": int(free0 - free1),
+                   "torch_peak_growth_bytes": int(torch.cuda.max_memory_allocated(dev) - alloc0),
+                   "backward_workspace_bytes": int(bws.numel()),
+                   "largest_segment": max(w2.seqlens_q),
+                   "score_matrix_bytes_if_materialised": 4 * max(w2.seqlens_q) ** 2 * 32}
         bflops = 2.5 * fwd_flops(w2.seqlens_q, 32, 128)
         btf = bflops / (bwd_ms * 1e-3) / 1e12
         peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -529,7 +544,8 @@ def run_ours(args, world, rank, local):
                                 "traffic": traffic_for("mea_bwd_dkdv_kernel"),
                                 "peak_kind": f"dense bf16 burst, {peak_src}",
                                 "kernel": "mea_bwd_pre_kernel + mea_bwd_dkdv_kernel + "
-                                          "mea_bwd_dq_kernel"}}
+                                          "mea_bwd_dq_kernel"},
+                   "memory": mem_obj}
 
     if rank != 0:
         return 0
