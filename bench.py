@@ -484,7 +484,9 @@ def run_ours(args, world, rank, local):
                      "value": aggregate_throughput(dbytes, world, pms) / 1e9, "unit": "GB/s",
                      "ms_per_call": pms, "block_size": pbs,
                      "roofline": {"bound": "hbm", "achieved": pgbs, "peak": hbm, "unit": "GB/s",
-                                  "frac": pgbs / hbm, "traffic": None,
+                                  "frac": pgbs / hbm,
+                                  "traffic": traffic_for("mea_decode_split_kernel_paged")
+                                  if pbs == 16 else None,
                                   "peak_kind": f"HBM copy bandwidth, {peak_src}",
                                   "kernel": "mea_decode_split_kernel<paged> + "
                                             "mea_lse_merge_kernel",
@@ -541,7 +543,7 @@ def run_ours(args, world, rank, local):
                    "launches_per_call": 3,
                    "roofline": {"bound": "tensor", "achieved": btf, "peak": peak,
                                 "unit": "TFLOP/s", "frac": btf / peak,
-                                "traffic": traffic_for("mea_bwd_dkdv_kernel"),
+                                "traffic": traffic_for("mea_backward_call"),
                                 "peak_kind": f"dense bf16 burst, {peak_src}",
                                 "kernel": "mea_bwd_pre_kernel + mea_bwd_dkdv_kernel + "
                                           "mea_bwd_dq_kernel"},
