@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-paged", dest="paged", action="store_false",
                     help="skip the paged-cache decode measurement")
+    ap.add_argument("--no-fp8", dest="fp8", action="store_false",
+                    help="skip the FP8 forward measurement")
     ap.add_argument("--paged-block-size", type=int, default=16,
                     help="slots per cache block of the paged decode measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -462,6 +464,43 @@ def run_ours(args, world, rank, local):
             if not do_fwd:
                 e2e.update({"value": e2e["decode_value"], "unit": "GB/s"})
 
+    # ---- FP8 forward on the packed prefill workload (e4m3 q/k/v), timed on its own
+    fp8_obj = None
+    if do_fwd and args.fp8:
+        q8 = (q.float() * 2.0).to(torch.float8_e4m3fn)
+        k8 = (k.float() * 4.0).to(torch.float8_e4m3fn)
+        v8 = (v.float() * 0.5).to(torch.float8_e4m3fn)
+        out8 = torch.empty_like(q)
+        lse8 = torch.empty_like(lse)
+
+        def fwd8():
+            mea.attention_packed_fp8(q8, k8, v8, cu, cu, max_q, causal=True, alibi_slopes=slopes,
+                                     scale=w2.scale, q_descale=0.5, k_descale=0.25,
+                                     v_descale=2.0, out=out8, lse=lse8)
+        for _ in range(args.warmup):
+            fwd8()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fwd8()
+        b.record(stream)
+        barrier(world)
+        f8ms = dist_max(a.elapsed_time(b), world) / args.steps
+        code = mea.device_error()
+        if code:
+            raise RuntimeError(f"device error word {code:#x} during the FP8 forward")
+        f8tf = flops / (f8ms * 1e-3) / 1e12
+        peak8 = 2.0 * pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        fp8_obj = {"metric": "attention fwd TFLOP/s, e4m3 inputs (packed causal GQA+ALiBi)",
+                   "value": aggregate_throughput(flops, world, f8ms) / 1e12, "unit": "TFLOP/s",
+                   "ms_per_call": f8ms, "dtype": "e4m3 in, bf16 out",
+                   "roofline": {"bound": "tensor", "achieved": f8tf, "peak": peak8,
+                                "unit": "TFLOP/s", "frac": f8tf / peak8, "traffic": None,
+                                "peak_kind": "dense fp8 = measured bf16 burst x 2 (nominal "
+                                             f"4.5 / 2.25 PFLOP/s), {peak_src}",
+                                "kernel": "mea_fwd_sm100_kernel<…, e4m3>"}}
+
     # ---- paged-cache decode of the same requests, timed on its own (not part of the step)
     paged_obj = None
     if do_dec and args.paged:
@@ -591,6 +630,8 @@ def run_ours(args, world, rank, local):
         if not do_fwd:
             line.update({"value": dec_obj["value"], "unit": "GB/s",
                          "roofline": dec_obj["roofline"]})
+    if fp8_obj is not None:
+        line["fp8_forward"] = fp8_obj
     if paged_obj is not None:
         line["paged_decode"] = paged_obj
     if bwd_obj is not None:

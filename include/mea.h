@@ -156,6 +156,26 @@ int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void
                                int split_keys, void* stream);
 
 /*
+ * mea_forward_fp8 — mea_forward with 8-bit e4m3 q, k, v (FP8 forward on the tensor cores).
+ *
+ * The inputs are e4m3 values (1 sign, 4 exponent, 3 mantissa bits, bias 7, largest finite 448,
+ * no infinities) with per-tensor descales: the attention is that of q_descale*q,
+ * k_descale*k, v_descale*v (exact products of the decoded values), with the same segments,
+ * masks, GQA grouping, ALiBi and scale as mea_forward. Q K^T accumulates in fp32; P is rounded
+ * to e4m3 for the P V product (its row sum and lse use the fp32 values); out is written in
+ * out_dtype (MEA_BF16 or MEA_F16), lse in fp32 natural log.
+ *   q, k, v   DEVICE e4m3 [total_q, n_heads_q, 128] / [total_k, n_heads_kv, 128].
+ *   head_dim  128 only (MEA_ERR_HEAD_DIM otherwise).
+ * Other arguments, errors and ownership as mea_forward.
+ */
+int mea_forward_fp8(const void* q, const void* k, const void* v, void* out, float* lse,
+                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int n_seqs,
+                    int total_q, int total_k, int max_seqlen_q, int n_heads_q, int n_heads_kv,
+                    int head_dim, float scale, int mask_kind, const float* alibi_slopes,
+                    float q_descale, float k_descale, float v_descale, int out_dtype,
+                    void* stream);
+
+/*
  * mea_backward_workspace_size — bytes of workspace mea_backward needs: one fp32 per (query head,
  * query token) for delta = rowsum(dout * out), plus 256 bytes of alignment slack.
  */

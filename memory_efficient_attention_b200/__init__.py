@@ -99,6 +99,40 @@ def attention_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out, lse
 
 
+def attention_packed_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, max_seqlen_q: int,
+                         causal: bool = False, alibi_slopes: Optional[torch.Tensor] = None,
+                         scale: Optional[float] = None, q_descale: float = 1.0,
+                         k_descale: float = 1.0, v_descale: float = 1.0,
+                         out_dtype: torch.dtype = torch.bfloat16,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """FP8 forward: q, k, v ``torch.float8_e4m3fn`` (D = 128) with per-tensor descales; returns
+    ``(out [T_q, Hq, D] out_dtype, lse [Hq, T_q] fp32)``."""
+    for t in (q, k, v):
+        if not t.is_cuda or t.dtype != torch.float8_e4m3fn:
+            raise MeaError(_lib.MEA_ERR_DTYPE, "q, k, v must be float8_e4m3fn on the GPU")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    tq, hq, d = q.shape
+    tk, hkv, _ = k.shape
+    n_seqs = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((tq, hq, d), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((hq, tq), dtype=torch.float32, device=q.device)
+    if alibi_slopes is not None:
+        alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
+    rc = _lib.load().mea_forward_fp8(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+        n_seqs, tq, tk, int(max_seqlen_q), hq, hkv, d, float(scale),
+        _lib.MEA_MASK_CAUSAL if causal else _lib.MEA_MASK_NONE, _ptr(alibi_slopes),
+        float(q_descale), float(k_descale), float(v_descale), _dtype_code(out.dtype),
+        _stream(q.device))
+    _lib.check(rc, "mea_forward_fp8")
+    return out, lse
+
+
 def backward_workspace_size(total_q: int, n_heads_q: int) -> int:
     return int(_lib.load().mea_backward_workspace_size(int(total_q), int(n_heads_q)))
 

@@ -29,7 +29,7 @@ MEA_MASK_NONE = 0
 MEA_MASK_CAUSAL = 1
 MEA_SELFTEST_WAIT_CODE = 0x7F01
 
-EXPORTS = ("mea_forward", "mea_backward_workspace_size", "mea_backward",
+EXPORTS = ("mea_forward", "mea_forward_fp8", "mea_backward_workspace_size", "mea_backward",
            "mea_decode_workspace_size", "mea_decode_splitkv", "mea_decode_paged",
            "mea_decode_splitkv_noalloc", "mea_status_string", "mea_device_error",
            "mea_set_wait_timeout_ns", "mea_wait_selftest", "mea_version")
@@ -50,6 +50,9 @@ def load() -> ctypes.CDLL:
     lib.mea_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci,
                                 vp, ci, vp]
     lib.mea_forward.restype = ci
+    lib.mea_forward_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf,
+                                    ci, vp, cf, cf, cf, ci, vp]
+    lib.mea_forward_fp8.restype = ci
     lib.mea_backward_workspace_size.argtypes = [ci, ci]
     lib.mea_backward_workspace_size.restype = sz
     lib.mea_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,

@@ -27,6 +27,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <type_traits>
 
@@ -49,22 +50,30 @@ struct FwdParams {
   int tok_per_tile;  // 128 / P tokens per sub-tile
   int t_max;         // max sub-tile pairs of a segment
   long long n_items; // t_max * n_seqs * n_hb
-  float c1;          // scale * log2(e)
+  float c1;          // scale * log2(e) (times the q and k descales for 8-bit inputs)
+  float o_scale;     // multiplies O before the division by l (the v descale; 1 for 16-bit)
   unsigned long long timeout_ns;
 };
 
-template <int D>
+// E8: q, k, v are 8-bit e4m3 (kind::f8f6f4 MMAs, P handed over as e4m3); otherwise 16-bit.
+template <int D, bool E8 = false>
 struct FwdCfg {
   static constexpr int BM = 128;
   static constexpr int BN = 128;
-  static constexpr int ATOMS = D / 64;  // 128-byte swizzle atoms along the head dim
+  static constexpr int ELEM = E8 ? 1 : 2;                // bytes per q/k/v element
+  static constexpr int ATOM_COLS = 128 / ELEM;           // elements per 128-byte swizzle row
+  static constexpr int ATOMS = D / ATOM_COLS;            // 128-byte swizzle atoms along D
+  static constexpr int KSTEP = 32 / ELEM;                // K elements per MMA (32 bytes)
+  static constexpr int P_COLS = 128 * ELEM / 4;          // TMEM columns holding P of one tile
   static constexpr uint32_t ATOM_BYTES = 128 * 128;
-  static constexpr uint32_t TILE_BYTES = 128 * D * 2;
-  static constexpr int NS = (D == 128) ? 5 : 8;
+  static constexpr uint32_t TILE_BYTES = 128 * D * ELEM;
+  static constexpr int NS = E8 ? 10 : ((D == 128) ? 5 : 8);
   static constexpr uint32_t SMEM_Q = 0;                 // two Q sub-tiles
   static constexpr uint32_t SMEM_KV = 2 * TILE_BYTES;
   static constexpr uint32_t SMEM_BAR = SMEM_KV + NS * TILE_BYTES;
-  static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
+  static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 512 + 1024;
+  static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
+  static_assert(!E8 || D == 128, "8-bit inputs: D = 128 (one 128-byte swizzle atom per row)");
   static constexpr int THREADS = 384;
   // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); warps 8-11
   // give theirs down to REGS_OTHER so that the two softmax warpgroups can take REGS_SOFTMAX.
@@ -169,10 +178,17 @@ __device__ __forceinline__ float tile_score_max(const float (&x)[128], float c1,
   }
 }
 
+// Two values as e4m3 (round to nearest even, saturating), the first in the low byte.
+__device__ __forceinline__ uint32_t fp8x2_e4m3(float lo, float hi) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE,
+                                                         __NV_E4M3));
+}
+
 // p(c) = 2^(c1*x(c) + slope2*c - off) (slope2 term only with ALiBi) for the 128 columns of this
-// thread's row, packed to 16-bit pairs and stored over the first 64 TMEM columns at t_s.
-// Returns the row sum of p in fp32 and, in emax, the largest exponent seen.
-template <bool BF16, bool ALIBI>
+// thread's row, packed to 16-bit pairs over the first 64 TMEM columns at t_s (E8: to e4m3
+// quadruples over the first 32 columns). Returns the row sum of p in fp32 and, in emax, the
+// largest exponent seen.
+template <bool BF16, bool ALIBI, bool E8 = false>
 __device__ __forceinline__ float exp_tile_to_tmem(const float (&x)[128], float c1, float slope2,
                                                   float off, uint32_t t_s, float& emax) {
   const uint64_t c1x2 = f2_pack(c1, c1);
@@ -198,9 +214,20 @@ __device__ __forceinline__ float exp_tile_to_tmem(const float (&x)[128], float c
       const float p0 = ex2_approx(e0);
       const float p1 = ex2_approx(e1);
       acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-      pk[i] = pack2<BF16>(p0, p1);
+      if constexpr (E8) {
+        const uint32_t two = fp8x2_e4m3(p0, p1);
+        if (i & 1)
+          pk[i >> 1] |= two << 16;
+        else
+          pk[i >> 1] = two;
+      } else {
+        pk[i] = pack2<BF16>(p0, p1);
+      }
     }
-    tmem_st16(t_s + c4 * 16, pk);
+    if constexpr (E8)
+      tmem_st8(t_s + c4 * 8, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
+    else
+      tmem_st16(t_s + c4 * 16, pk);
   }
   emax = fmaxf(m0, m1);
   const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
@@ -221,12 +248,14 @@ __device__ __forceinline__ void fwd_teardown(bool owner, uint32_t tmem, uint32_t
   }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool ALIBI>
+// BF16 selects the 16-bit type of q/k/v/out (bf16 or f16); with E8, q/k/v are e4m3 and out is
+// the BF16-selected 16-bit type.
+template <int D, bool BF16, bool CAUSAL, bool ALIBI, bool E8 = false>
 __global__ void __launch_bounds__(384, 1)
     mea_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, E8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -237,6 +266,7 @@ __global__ void __launch_bounds__(384, 1)
   constexpr int B_QF = 0, B_QE = 1, B_KVF = 2, B_KVE = 2 + C::NS, B_SF = 2 + 2 * C::NS;
   constexpr int B_PF = B_SF + 2, B_OF = B_PF + 2, B_OE = B_OF + 2, B_DR = B_OE + 2;
   constexpr int N_BARS = B_DR + 1;
+  static_assert(8 * N_BARS + 8 <= 512, "barrier region");
   const uint32_t bar0 = sbase + C::SMEM_BAR;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_BAR + 8 * N_BARS);
@@ -298,7 +328,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int a = 0; a < C::ATOMS; ++a)
-            tma_load_3d(q_s + h * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_q, BAR(B_QF), a * 64,
+            tma_load_3d(q_s + h * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_q, BAR(B_QF),
+                        a * C::ATOM_COLS,
                         it.hb * p.P, it.q0 + it.tok0 + h * p.tok_per_tile);
         ++q_cnt;
         for (int j = 0; j < nmax && ok; ++j) {
@@ -312,7 +343,8 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t dst = kv_s0 + s * C::TILE_BYTES;
 #pragma unroll
             for (int a = 0; a < C::ATOMS; ++a)
-              tma_load_3d(dst + a * C::ATOM_BYTES, w ? &tm_v : &tm_k, BAR(B_KVF + s), a * 64, g,
+              tma_load_3d(dst + a * C::ATOM_BYTES, w ? &tm_v : &tm_k, BAR(B_KVF + s),
+                          a * C::ATOM_COLS, g,
                           it.k0 + (nmax - 1 - j) * 128);
             ++kv_cnt;
           }
@@ -334,8 +366,10 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 8) {
     // ---------------------------------------------------------------- tcgen05 issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_QK = umma_idesc_f16(BF16, 128, 128, false, false);
-      constexpr uint32_t IDESC_PV = umma_idesc_f16(BF16, 128, D, false, true);
+      constexpr uint32_t IDESC_QK = E8 ? umma_idesc_e4m3(128, 128, false, false)
+                                       : umma_idesc_f16(BF16, 128, 128, false, false);
+      constexpr uint32_t IDESC_PV = E8 ? umma_idesc_e4m3(128, D, false, true)
+                                       : umma_idesc_f16(BF16, 128, D, false, true);
       uint32_t kv_cnt = 0, q_cnt = 0;
       uint32_t pv_cnt[2] = {0, 0}, oe_cnt[2] = {0, 0};
       bool ok = true;
@@ -381,9 +415,11 @@ __global__ void __launch_bounds__(384, 1)
               tc_fence_after();
               const uint32_t vbase = kv_s0 + vs * C::TILE_BYTES;
 #pragma unroll
-              for (int kk = 0; kk < C::BN / 16; ++kk) {
-                const uint64_t bd = umma_desc_sw128(vbase + kk * 2048, C::ATOM_BYTES, 1024);
-                mma_ts(tmem + C::TM_O + h * D, tmem + h * 128 + kk * 8, bd, IDESC_PV,
+              for (int kk = 0; kk < C::BN / C::KSTEP; ++kk) {
+                // V rows kk*KSTEP.. (128-byte rows), P columns kk*8.. (32 bytes per row)
+                const uint64_t bd =
+                    umma_desc_sw128(vbase + kk * C::KSTEP * 128, C::ATOM_BYTES, 1024);
+                mma_ts_k<E8>(tmem + C::TM_O + h * D, tmem + h * 128 + kk * 8, bd, IDESC_PV,
                        (j == first_h + 1 && kk == 0) ? 0u : 1u);
               }
               ++pv_cnt[h];
@@ -394,11 +430,11 @@ __global__ void __launch_bounds__(384, 1)
               const uint32_t kbase = kv_s0 + ks * C::TILE_BYTES;
               const uint32_t qbase = q_s + h * C::TILE_BYTES;
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
+              for (int kk = 0; kk < D / C::KSTEP; ++kk) {
                 const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
                 const uint64_t ad = umma_desc_sw128(qbase + off, 16, 1024);
                 const uint64_t bd = umma_desc_sw128(kbase + off, 16, 1024);
-                mma_ss(tmem + h * 128, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+                mma_ss_k<E8>(tmem + h * 128, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
               }
               mma_commit(BAR(B_SF + h));
             }
@@ -507,7 +543,8 @@ __global__ void __launch_bounds__(384, 1)
           }
           const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
           float emax;
-          float rs = exp_tile_to_tmem<BF16, ALIBI>(x, p.c1, slope2, m_use - kconst, t_s, emax);
+          float rs =
+              exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_use - kconst, t_s, emax);
           if (speculate) {
             const bool over = emax > 8.0f;
             if (__any_sync(0xffffffffu, over)) {
@@ -518,7 +555,8 @@ __global__ void __launch_bounds__(384, 1)
                 l *= alpha;
                 m_ref = m_tile;
               }
-              rs = exp_tile_to_tmem<BF16, ALIBI>(x, p.c1, slope2, m_ref - kconst, t_s, emax);
+              rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_ref - kconst, t_s,
+                                                     emax);
             }
           }
           l += rs;
@@ -541,7 +579,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
           float unused;
-          l += exp_tile_to_tmem<BF16, false>(x, 1.f, 0.f, m_use, t_s, unused);
+          l += exp_tile_to_tmem<BF16, false, E8>(x, 1.f, 0.f, m_use, t_s, unused);
         }
         // O_h holds the tiles visited before this one and its last PV has completed (it was
         // issued before this QK).
@@ -568,7 +606,7 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) break;
       ++ocnt;
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = l > 0.f ? p.o_scale / l : 0.f;
 #pragma unroll 1
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t o[32];

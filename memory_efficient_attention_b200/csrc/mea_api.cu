@@ -62,16 +62,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 3-D tiled map over a row-major [d2, d1, d0] tensor of 16-bit elements, 128-byte swizzle.
+constexpr int kDtypeE4M3 = 2;  // internal: 8-bit e4m3 tensor (mea_forward_fp8)
+
 bool encode_3d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
                uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const uint64_t es = dtype == kDtypeE4M3 ? 1 : 2;
   cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
   cuuint32_t box[3] = {b0, b1, b2};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, dtype == MEA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+  CUresult r = fn(map, dtype == kDtypeE4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                       : dtype == MEA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                   3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -89,11 +93,11 @@ int largest_pow2_divisor(int x, int cap) {
 // ------------------------------------------------------------------------------------------
 // Forward launch dispatch.
 // ------------------------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL, bool ALIBI>
+template <int D, bool BF16, bool CAUSAL, bool ALIBI, bool E8 = false>
 int launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const mea::FwdParams& p, int grid, cudaStream_t stream) {
-  auto kern = mea::mea_fwd_sm100_kernel<D, BF16, CAUSAL, ALIBI>;
-  constexpr uint32_t smem = mea::FwdCfg<D>::SMEM_TOTAL;
+  auto kern = mea::mea_fwd_sm100_kernel<D, BF16, CAUSAL, ALIBI, E8>;
+  constexpr uint32_t smem = mea::FwdCfg<D, E8>::SMEM_TOTAL;
   static std::once_flag once[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -106,14 +110,14 @@ int launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool E8 = false>
 int launch_fwd_d(bool causal, bool alibi, const CUtensorMap& tq, const CUtensorMap& tk,
                  const CUtensorMap& tv, const mea::FwdParams& p, int grid, cudaStream_t s) {
   if (causal)
-    return alibi ? launch_fwd_t<D, BF16, true, true>(tq, tk, tv, p, grid, s)
-                 : launch_fwd_t<D, BF16, true, false>(tq, tk, tv, p, grid, s);
-  return alibi ? launch_fwd_t<D, BF16, false, true>(tq, tk, tv, p, grid, s)
-               : launch_fwd_t<D, BF16, false, false>(tq, tk, tv, p, grid, s);
+    return alibi ? launch_fwd_t<D, BF16, true, true, E8>(tq, tk, tv, p, grid, s)
+                 : launch_fwd_t<D, BF16, true, false, E8>(tq, tk, tv, p, grid, s);
+  return alibi ? launch_fwd_t<D, BF16, false, true, E8>(tq, tk, tv, p, grid, s)
+               : launch_fwd_t<D, BF16, false, false, E8>(tq, tk, tv, p, grid, s);
 }
 
 // 4-D tiled map over a paged cache [d3 blocks, d2 slots, d1 heads, d0] of 16-bit elements.
@@ -297,6 +301,74 @@ __global__ void mea_wait_selftest_kernel(unsigned long long timeout_ns, int arri
 }
 }  // namespace mea
 
+// dtype: the 16-bit type of out (and of q, k, v unless e8); e8: q, k, v are e4m3 with descales
+// qk_descale (folded into the exponent) and v_descale (applied to O before the division by l).
+int forward_impl(const void* q, const void* k, const void* v, void* out, float* lse,
+                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int n_seqs,
+                 int total_q, int total_k, int max_seqlen_q, int n_heads_q, int n_heads_kv,
+                 int head_dim, float scale, int mask_kind, const float* alibi_slopes, int dtype,
+                 bool e8, float qk_descale, float v_descale, void* stream) {
+  if (!q || !k || !v || !out || !cu_seqlens_q || !cu_seqlens_k) return MEA_ERR_NULL;
+  if (n_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_q > total_q)
+    return MEA_ERR_SHAPE;
+  if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
+  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (e8 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
+  if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
+  if (!std::isfinite(scale) || !std::isfinite(qk_descale) || !std::isfinite(v_descale))
+    return MEA_ERR_SCALE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
+      (alibi_slopes && !aligned(alibi_slopes, 4)))
+    return MEA_ERR_ALIGN;
+  DeviceInfo di;
+  if (int rc = current_device_info(di); rc != MEA_OK) return rc;
+  if (total_q == 0 || max_seqlen_q == 0) return MEA_OK;
+
+  const int R = n_heads_q / n_heads_kv;
+  const int P = largest_pow2_divisor(R, 128);
+  mea::FwdParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.slopes = alibi_slopes;
+  p.n_seqs = n_seqs;
+  p.total_q = total_q;
+  p.hq = n_heads_q;
+  p.P = P;
+  p.R = R;
+  p.n_hb = n_heads_q / P;
+  p.tok_per_tile = 128 / P;
+  p.t_max = (max_seqlen_q + 2 * p.tok_per_tile - 1) / (2 * p.tok_per_tile);
+  p.n_items = static_cast<long long>(p.t_max) * n_seqs * p.n_hb;
+  p.c1 = scale * qk_descale * 1.4426950408889634f;
+  p.o_scale = v_descale;
+  p.timeout_ns = g_timeout_ns.load();
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t tk_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
+  const int in_dtype = e8 ? kDtypeE4M3 : dtype;
+  const uint32_t box0 = e8 ? 128 : 64;  // elements per 128-byte swizzle row
+  if (!encode_3d(&tq, q, in_dtype, head_dim, n_heads_q, total_q, box0, P, 128 / P) ||
+      !encode_3d(&tk, k, in_dtype, head_dim, n_heads_kv, tk_rows, box0, 1, 128) ||
+      !encode_3d(&tv, v, in_dtype, head_dim, n_heads_kv, tk_rows, box0, 1, 128))
+    return MEA_ERR_CUDA;
+  const int grid = static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool causal = mask_kind == MEA_MASK_CAUSAL;
+  const bool alibi = alibi_slopes != nullptr;
+  if (e8)
+    return dtype == MEA_BF16 ? launch_fwd_d<128, true, true>(causal, alibi, tq, tk, tv, p, grid, s)
+                             : launch_fwd_d<128, false, true>(causal, alibi, tq, tk, tv, p, grid, s);
+  if (head_dim == 128)
+    return dtype == MEA_BF16 ? launch_fwd_d<128, true>(causal, alibi, tq, tk, tv, p, grid, s)
+                             : launch_fwd_d<128, false>(causal, alibi, tq, tk, tv, p, grid, s);
+  return dtype == MEA_BF16 ? launch_fwd_d<64, true>(causal, alibi, tq, tk, tv, p, grid, s)
+                           : launch_fwd_d<64, false>(causal, alibi, tq, tk, tv, p, grid, s);
+}
+
 extern "C" {
 
 const char* mea_version(void) { return "mea 0.1.0 (sm_100a)"; }
@@ -419,57 +491,20 @@ int mea_forward(const void* q, const void* k, const void* v, void* out, float* l
                 int total_q, int total_k, int max_seqlen_q, int n_heads_q, int n_heads_kv,
                 int head_dim, float scale, int mask_kind, const float* alibi_slopes, int dtype,
                 void* stream) {
-  if (!q || !k || !v || !out || !cu_seqlens_q || !cu_seqlens_k) return MEA_ERR_NULL;
-  if (n_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_q > total_q)
-    return MEA_ERR_SHAPE;
-  if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
-  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
-  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
-  if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
-  if (!std::isfinite(scale)) return MEA_ERR_SCALE;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
-      (lse && !aligned(lse, 4)) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
-      (alibi_slopes && !aligned(alibi_slopes, 4)))
-    return MEA_ERR_ALIGN;
-  DeviceInfo di;
-  if (int rc = current_device_info(di); rc != MEA_OK) return rc;
-  if (total_q == 0 || max_seqlen_q == 0) return MEA_OK;
+  return forward_impl(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, n_seqs, total_q, total_k,
+                      max_seqlen_q, n_heads_q, n_heads_kv, head_dim, scale, mask_kind,
+                      alibi_slopes, dtype, false, 1.f, 1.f, stream);
+}
 
-  const int R = n_heads_q / n_heads_kv;
-  const int P = largest_pow2_divisor(R, 128);
-  mea::FwdParams p{};
-  p.out = out;
-  p.lse = lse;
-  p.cu_q = cu_seqlens_q;
-  p.cu_k = cu_seqlens_k;
-  p.slopes = alibi_slopes;
-  p.n_seqs = n_seqs;
-  p.total_q = total_q;
-  p.hq = n_heads_q;
-  p.P = P;
-  p.R = R;
-  p.n_hb = n_heads_q / P;
-  p.tok_per_tile = 128 / P;
-  p.t_max = (max_seqlen_q + 2 * p.tok_per_tile - 1) / (2 * p.tok_per_tile);
-  p.n_items = static_cast<long long>(p.t_max) * n_seqs * p.n_hb;
-  p.c1 = scale * 1.4426950408889634f;
-  p.timeout_ns = g_timeout_ns.load();
-
-  CUtensorMap tq, tk, tv;
-  const uint64_t tk_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
-  if (!encode_3d(&tq, q, dtype, head_dim, n_heads_q, total_q, 64, P, 128 / P) ||
-      !encode_3d(&tk, k, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 128) ||
-      !encode_3d(&tv, v, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 128))
-    return MEA_ERR_CUDA;
-  const int grid = static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool causal = mask_kind == MEA_MASK_CAUSAL;
-  const bool alibi = alibi_slopes != nullptr;
-  if (head_dim == 128)
-    return dtype == MEA_BF16 ? launch_fwd_d<128, true>(causal, alibi, tq, tk, tv, p, grid, s)
-                             : launch_fwd_d<128, false>(causal, alibi, tq, tk, tv, p, grid, s);
-  return dtype == MEA_BF16 ? launch_fwd_d<64, true>(causal, alibi, tq, tk, tv, p, grid, s)
-                           : launch_fwd_d<64, false>(causal, alibi, tq, tk, tv, p, grid, s);
+int mea_forward_fp8(const void* q, const void* k, const void* v, void* out, float* lse,
+                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int n_seqs,
+                    int total_q, int total_k, int max_seqlen_q, int n_heads_q, int n_heads_kv,
+                    int head_dim, float scale, int mask_kind, const float* alibi_slopes,
+                    float q_descale, float k_descale, float v_descale, int out_dtype,
+                    void* stream) {
+  return forward_impl(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, n_seqs, total_q, total_k,
+                      max_seqlen_q, n_heads_q, n_heads_kv, head_dim, scale, mask_kind,
+                      alibi_slopes, out_dtype, true, q_descale * k_descale, v_descale, stream);
 }
 
 size_t mea_decode_workspace_size(int n_seqs, int total_k, int n_heads_q, int n_heads_kv,

@@ -15,6 +15,7 @@ from .core import (  # noqa: F401
     attention_probs,
     attention_rows,
     decode,
+    e4m3_decode,
     lse_merge,
     paged_gather,
     segment_positions,

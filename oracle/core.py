@@ -63,6 +63,7 @@ __all__ = [
     "attention_bruteforce",
     "attention_backward",
     "paged_gather",
+    "e4m3_decode",
 ]
 
 F64 = torch.float64
@@ -374,3 +375,20 @@ def paged_gather(cache: torch.Tensor, block_table, seqlens_k: Sequence[int]) -> 
     if not rows:
         return cache.new_zeros((0,) + tuple(cache.shape[2:]))
     return torch.stack(rows)
+
+
+def e4m3_decode(codes: torch.Tensor) -> torch.Tensor:
+    """Values of 8-bit E4M3 codes (uint8) in float64, from the format's definition: sign bit 7,
+    exponent bits 6..3 with bias 7, mantissa bits 2..0; exponent field 0 is subnormal
+    (m/8 * 2^-6); the all-ones exponent with mantissa 7 is NaN (no infinities); largest finite
+    value 448. The FP8 forward's attention is this oracle's attention of the decoded values times
+    the per-tensor descales ([zizhi §3] "混合精度计算流水线" lists FP8 among the supported
+    precisions, with the critical parts of the computation kept in higher precision)."""
+    c = codes.to(torch.int64)
+    sign = torch.where((c >> 7) & 1 == 1, -1.0, 1.0).to(F64)
+    e = (c >> 3) & 0xF
+    m = (c & 7).to(F64)
+    normal = torch.ldexp(1.0 + m / 8.0, (e - 7).to(torch.int64).to(torch.int32)).to(F64)
+    sub = m / 8.0 * 2.0 ** -6
+    val = torch.where(e == 0, sub, normal) * sign
+    return torch.where((e == 15) & ((c & 7) == 7), torch.full_like(val, float("nan")), val)

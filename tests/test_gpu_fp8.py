@@ -1,0 +1,105 @@
+"""GPU parity of the FP8 forward (mea_forward_fp8 through the C ABI) against the float64 oracle.
+
+Inputs: seeded N(0,1) values divided by their descale and rounded to e4m3; the oracle is the
+attention of the decoded values (oracle.e4m3_decode, pinned to the format definition) times the
+descales, in float64.
+
+Tolerance, from the arithmetic: the scores are exact products of e4m3 values summed in fp32;
+the only rounding of consequence is P to e4m3 before P V (relative error <= 2^-4 for normal
+values, absolute <= 2^-10 for subnormals in the kernel's units, which are never smaller than the
+row-max-normalised ones), then out to bf16/f16. Per element, with pi the oracle's softmax
+probabilities of the row:
+    |out - ref| <= sum_j max(2^-4 pi_ij, 2^-10 max_j pi_ij) |v_j| + 2^-8 |ref| + 1e-5,
+and |lse - lse_ref| <= 1e-3 (it uses the fp32 P).
+"""
+import math
+
+import pytest
+import torch
+
+import memory_efficient_attention_b200 as mea
+import oracle
+from mea_workloads import alibi_slope_values, cu_seqlens, randn
+
+pytestmark = pytest.mark.gpu
+
+QD, KD, VD = 0.5, 0.25, 2.0   # per-tensor descales
+
+
+def _quantized(shape, seed, descale):
+    x = randn(shape, seed, torch.float32) / descale
+    return x.to(torch.float8_e4m3fn)
+
+
+def _case(seqlens, hq, hkv, causal, alibi, scale, seed, out_dtype=torch.bfloat16):
+    tq = sum(seqlens)
+    q8 = _quantized((tq, hq, 128), seed, QD)
+    k8 = _quantized((tq, hkv, 128), seed + 1, KD)
+    v8 = _quantized((tq, hkv, 128), seed + 2, VD)
+    slopes = alibi_slope_values(hq) if alibi else None
+    cu = cu_seqlens(seqlens)
+    out, lse = mea.attention_packed_fp8(q8.cuda(), k8.cuda(), v8.cuda(), cu.cuda(), cu.cuda(),
+                                        max(seqlens), causal=causal,
+                                        alibi_slopes=None if slopes is None else slopes.cuda(),
+                                        scale=scale, q_descale=QD, k_descale=KD, v_descale=VD,
+                                        out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert mea.device_error() == 0
+    q = oracle.e4m3_decode(q8.view(torch.uint8)) * QD
+    k = oracle.e4m3_decode(k8.view(torch.uint8)) * KD
+    v = oracle.e4m3_decode(v8.view(torch.uint8)) * VD
+    sl = None if slopes is None else slopes.double()
+    ref, lref = oracle.attention(q, k, v, cu.tolist(), cu.tolist(), scale, causal, sl)
+    probs = oracle.attention_probs(q, k, v, cu.tolist(), cu.tolist(), scale, causal, sl)
+    r = hq // hkv
+    bound = torch.zeros_like(ref)
+    c = cu.tolist()
+    for s, pr in enumerate(probs):            # pr [Hq, L, L]
+        if pr.numel() == 0:
+            continue
+        pmax = pr.amax(dim=-1, keepdim=True)
+        w = torch.maximum(2.0 ** -4 * pr, 2.0 ** -10 * pmax)
+        for h in range(hq):
+            va = v[c[s]:c[s + 1], h // r].abs()
+            bound[c[s]:c[s + 1], h] = w[h] @ va
+    bound = bound + 2.0 ** -8 * ref.abs() + 1e-5
+    o = out.cpu().double()
+    assert torch.isfinite(o).all()
+    err = (o - ref).abs()
+    worst = float((err - bound).max())
+    assert worst <= 0.0, f"max err {float(err.max()):.3e}, exceeds the bound by {worst:.3e}"
+    fin = torch.isfinite(lref)
+    lg = lse.cpu().double()
+    assert torch.equal(torch.isfinite(lg), fin)
+    assert float((lg[fin] - lref[fin]).abs().max()) <= 1e-3
+    return float(err.max()), float((err / bound).max())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("alibi", [False, True])
+def test_fp8_packed_varlen(causal, alibi):
+    _case([37, 120, 8, 200], 8, 2, causal, alibi, 1 / math.sqrt(128), 1500)
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (64, 8), (8, 8), (6, 2)])
+def test_fp8_gqa_packing(hq, hkv):
+    _case([130, 77, 300], hq, hkv, True, True, 0.088, 1510 + hq)
+
+
+@pytest.mark.parametrize("lens", [[1], [128], [129], [255, 1, 257]])
+def test_fp8_tile_edges(lens):
+    _case(lens, 8, 4, True, False, 0.1, 1520 + sum(lens))
+
+
+def test_fp8_half_output_and_longer_segments():
+    _case([1000, 700], 8, 2, True, True, 1 / math.sqrt(128), 1530, out_dtype=torch.float16)
+
+
+def test_fp8_rejects_other_head_dims_and_dtypes():
+    x = torch.zeros((4, 2, 64), dtype=torch.float8_e4m3fn, device="cuda")
+    cu = torch.tensor([0, 4], dtype=torch.int32, device="cuda")
+    with pytest.raises(mea.MeaError):
+        mea.attention_packed_fp8(x, x, x, cu, cu, 4)
+    y = torch.zeros((4, 2, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(mea.MeaError):
+        mea.attention_packed_fp8(y, y, y, cu, cu, 4)

@@ -435,3 +435,21 @@ def test_paged_gather_inverts_a_brute_force_scatter():
             off += length
         back = oracle.paged_gather(cache, table, lens)
         assert torch.equal(back, packed)
+
+
+def test_e4m3_decode_matches_the_format_definition_and_torch():
+    """E4M3 code points worked out by hand from the format (sign, 4-bit exponent bias 7, 3-bit
+    mantissa, subnormals, no infinities), and agreement with torch's float8_e4m3fn decoding
+    over all 256 codes (NaN codes 0x7F / 0xFF excepted)."""
+    by_hand = {0x00: 0.0, 0x38: 1.0, 0x40: 2.0, 0x3C: 1.5, 0x7E: 448.0, 0xFE: -448.0,
+               0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x30: 0.5, 0xB8: -1.0}
+    codes = torch.tensor(list(by_hand), dtype=torch.uint8)
+    got = oracle.e4m3_decode(codes)
+    for c, want in zip(by_hand, got.tolist()):
+        assert want == by_hand[c], hex(c)
+    allc = torch.arange(256, dtype=torch.uint8)
+    dec = oracle.e4m3_decode(allc)
+    assert torch.isnan(dec[0x7F]) and torch.isnan(dec[0xFF])
+    tv = allc.view(torch.float8_e4m3fn).to(F64)
+    ok = ~torch.isnan(dec)
+    assert torch.equal(dec[ok], tv[ok])
