@@ -25,8 +25,9 @@ from . import _lib
 from ._lib import MeaError  # noqa: F401
 
 __all__ = [
-    "memory_efficient_attention", "attention_packed", "decode_splitkv", "decode_splitkv_noalloc",
-    "decode_workspace_size", "alibi_slopes", "BlockDiagonalMask", "BlockDiagonalCausalMask",
+    "memory_efficient_attention", "attention_packed", "attention_packed_fp8",
+    "attention_packed_backward", "backward_workspace_size", "decode_splitkv", "decode_paged",
+    "decode_splitkv_noalloc", "decode_workspace_size", "wait_selftest", "alibi_slopes", "BlockDiagonalMask", "BlockDiagonalCausalMask",
     "LowerTriangularMask", "device_error", "set_wait_timeout_ns", "MeaError", "library_path",
 ]
 
