@@ -13,6 +13,7 @@
 
 #include "../../include/mea.h"
 #include "bwd_sm100.cuh"
+#include "bwd_tc_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "ptx.cuh"
@@ -151,32 +152,40 @@ bool set_smem_once(K kern, uint32_t smem, std::once_flag (&once)[kMaxDevices]) {
   return err == cudaSuccess;
 }
 
+struct BwdMaps {
+  CUtensorMap q, dout, k, v;  // 128-row boxes of one head
+};
+
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
-int launch_bwd_t(const mea::BwdParams& p, int max_q, int max_k, cudaStream_t stream) {
-  constexpr uint32_t smem = mea::BwdCfg<D>::SMEM;
-  auto kdkdv = mea::mea_bwd_dkdv_kernel<D, BF16, CAUSAL, ALIBI>;
-  auto kdq = mea::mea_bwd_dq_kernel<D, BF16, CAUSAL, ALIBI>;
+int launch_bwd_t(const BwdMaps& m, const mea::BwdParams& p, int max_q, int max_k,
+                 cudaStream_t stream) {
+  constexpr uint32_t smem = mea::BwdTcCfg<D>::SMEM_TOTAL;
+  auto kdkdv = mea::mea_bwd_dkdv_tc_kernel<D, BF16, CAUSAL, ALIBI>;
+  auto kdq = mea::mea_bwd_dq_tc_kernel<D, BF16, CAUSAL, ALIBI>;
   static std::once_flag once_a[kMaxDevices], once_b[kMaxDevices];
   if (!set_smem_once(kdkdv, smem, once_a) || !set_smem_once(kdq, smem, once_b))
     return MEA_ERR_CUDA;
+  const unsigned long long tmo = g_timeout_ns.load();
   const long long rows = static_cast<long long>(p.total_q) * p.hq;
   if (rows > 0)
     mea::mea_bwd_pre_kernel<D, BF16><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(p);
   if (max_k > 0)
-    kdkdv<<<dim3((max_k + 63) / 64, p.n_seqs, p.hkv), 128, smem, stream>>>(p);
+    kdkdv<<<dim3((max_k + 127) / 128, p.n_seqs, p.hkv), mea::BwdTcCfg<D>::THREADS, smem,
+            stream>>>(m.q, m.dout, m.k, m.v, p, tmo);
   if (max_q > 0)
-    kdq<<<dim3((max_q + 63) / 64, p.n_seqs, p.hq), 128, smem, stream>>>(p);
+    kdq<<<dim3((max_q + 127) / 128, p.n_seqs, p.hq), mea::BwdTcCfg<D>::THREADS, smem,
+          stream>>>(m.q, m.dout, m.k, m.v, p, tmo);
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
 
 template <int D, bool BF16>
-int launch_bwd_d(bool causal, bool alibi, const mea::BwdParams& p, int mq, int mk,
-                 cudaStream_t s) {
+int launch_bwd_d(bool causal, bool alibi, const BwdMaps& m, const mea::BwdParams& p, int mq,
+                 int mk, cudaStream_t s) {
   if (causal)
-    return alibi ? launch_bwd_t<D, BF16, true, true>(p, mq, mk, s)
-                 : launch_bwd_t<D, BF16, true, false>(p, mq, mk, s);
-  return alibi ? launch_bwd_t<D, BF16, false, true>(p, mq, mk, s)
-               : launch_bwd_t<D, BF16, false, false>(p, mq, mk, s);
+    return alibi ? launch_bwd_t<D, BF16, true, true>(m, p, mq, mk, s)
+                 : launch_bwd_t<D, BF16, true, false>(m, p, mq, mk, s);
+  return alibi ? launch_bwd_t<D, BF16, false, true>(m, p, mq, mk, s)
+               : launch_bwd_t<D, BF16, false, false>(m, p, mq, mk, s);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -474,16 +483,24 @@ int mea_backward(const void* q, const void* k, const void* v, const void* out, c
   p.R = n_heads_q / n_heads_kv;
   p.scale = scale;
   p.c1 = scale * 1.4426950408889634f;
+  BwdMaps m;
+  const uint64_t tq_rows = total_q > 0 ? static_cast<uint64_t>(total_q) : 1;
+  const uint64_t tk_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
+  if (!encode_3d(&m.q, q, dtype, head_dim, n_heads_q, tq_rows, 64, 1, 128) ||
+      !encode_3d(&m.dout, dout, dtype, head_dim, n_heads_q, tq_rows, 64, 1, 128) ||
+      !encode_3d(&m.k, k, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 128) ||
+      !encode_3d(&m.v, v, dtype, head_dim, n_heads_kv, tk_rows, 64, 1, 128))
+    return MEA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool causal = mask_kind == MEA_MASK_CAUSAL;
   const bool alibi = alibi_slopes != nullptr;
   if (head_dim == 128)
     return dtype == MEA_BF16
-               ? launch_bwd_d<128, true>(causal, alibi, p, max_seqlen_q, max_seqlen_k, s)
-               : launch_bwd_d<128, false>(causal, alibi, p, max_seqlen_q, max_seqlen_k, s);
+               ? launch_bwd_d<128, true>(causal, alibi, m, p, max_seqlen_q, max_seqlen_k, s)
+               : launch_bwd_d<128, false>(causal, alibi, m, p, max_seqlen_q, max_seqlen_k, s);
   return dtype == MEA_BF16
-             ? launch_bwd_d<64, true>(causal, alibi, p, max_seqlen_q, max_seqlen_k, s)
-             : launch_bwd_d<64, false>(causal, alibi, p, max_seqlen_q, max_seqlen_k, s);
+             ? launch_bwd_d<64, true>(causal, alibi, m, p, max_seqlen_q, max_seqlen_k, s)
+             : launch_bwd_d<64, false>(causal, alibi, m, p, max_seqlen_q, max_seqlen_k, s);
 }
 
 int mea_forward(const void* q, const void* k, const void* v, void* out, float* lse,

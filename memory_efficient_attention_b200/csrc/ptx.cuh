@@ -17,7 +17,7 @@ namespace mea {
 // ------------------------------------------------------------------------------------------
 __device__ unsigned int g_mea_error = 0;
 
-enum : unsigned { KID_FWD = 1, KID_DECODE = 2, KID_MERGE = 3 };
+enum : unsigned { KID_FWD = 1, KID_DECODE = 2, KID_MERGE = 3, KID_BWD = 4 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
