@@ -20,8 +20,10 @@
 // tiles the rows see: S = Q K^T, dP = dO V^T, dS (thread = row), dQ += dS K.
 // TMEM: S [0,128), dP [128,256), dQ [256,256+D).
 //
-// Roles (192 threads): warps 0-3 elementwise + epilogue, warp 4 tcgen05 issuer (owns TMEM),
-// warp 5 TMA producer. Every wait is bounded; no named barriers inside the role loops.
+// Roles (320 threads): two elementwise warpgroups (warps 0-3 and 4-7; thread = TMEM lane; group
+// w handles columns [64w, 64w+64) of the 128-column S/dP tiles and writes its packed P / dS over
+// the first 32 of them, so the groups never touch each other's columns), warp 8 tcgen05 issuer
+// (owns TMEM), warp 9 TMA producer. Every wait is bounded; no named barriers in the role loops.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -45,7 +47,12 @@ struct BwdTcCfg {
   static constexpr uint32_t SMEM_BAR = SMEM_RING + 4 * TILE_BYTES;
   static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
   static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
+  // Column of the packed 16-bit operand for 16-row step k16 of a 128-column tile: group k16/4
+  // wrote rows 64*(k16/4).. at its own columns 64*(k16/4) + [0, 32).
+  __device__ static constexpr uint32_t packed_col(int k16) {
+    return static_cast<uint32_t>(64 * (k16 >> 2) + (k16 & 3) * 8);
+  }
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
@@ -56,7 +63,7 @@ __device__ __forceinline__ uint32_t bpack2(float lo, float hi) {
 
 // -------------------------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     mea_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_do,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -97,13 +104,13 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(TBAR(B_QE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
-    mbar_init(TBAR(B_PF), 128);
+    mbar_init(TBAR(B_PF), 256);
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -113,7 +120,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
 
-  if (warp == 5) {
+  if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t loaded = 0;
@@ -147,7 +154,7 @@ __global__ void __launch_bounds__(192, 1)
       for (uint32_t it = (loaded > 2 ? loaded - 2 : 0); it < loaded; ++it)
         mbar_wait(TBAR(B_QF + (it & 1)), (it >> 1) & 1, &never, tmo, ecode | 15);
     }
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
       constexpr uint32_t ID_KK = umma_idesc_f16(BF16, 128, 128, false, false);  // both K-major
@@ -170,12 +177,12 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t dos = qs + C::TILE_BYTES;
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16)
-            mma_ts(tmem + T_DV, tmem + T_S + k16 * 8,
+            mma_ts(tmem + T_DV, tmem + T_S + C::packed_col(k16),
                    umma_desc_sw128(dos + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
                    (it - 1 > 0 || k16 > 0) ? 1u : 0u);
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16)
-            mma_ts(tmem + T_DK, tmem + T_DP + k16 * 8,
+            mma_ts(tmem + T_DK, tmem + T_DP + C::packed_col(k16),
                    umma_desc_sw128(qs + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
                    (it - 1 > 0 || k16 > 0) ? 1u : 0u);
           mma_commit(TBAR(B_QE + ((it - 1) & 1)));
@@ -206,9 +213,10 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ elementwise (thread = key)
-    const int kl = threadIdx.x;                         // key within the tile = TMEM lane
+    const int wg = threadIdx.x >> 7;                    // column half of this warpgroup
+    const int kl = threadIdx.x & 127;                   // key within the tile = TMEM lane
     const int key = key0 + kl;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       ok = mbar_wait(TBAR(B_SF), it & 1, abort_flag, tmo, ecode | 5);
@@ -221,7 +229,8 @@ __global__ void __launch_bounds__(192, 1)
       float slope2 = 0.f;
       if constexpr (ALIBI) slope2 = __ldg(p.slopes + h) * LOG2E;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * wg + cc;            // 32-column chunk of the tile
         uint32_t sv[32], dv[32];
         tmem_ld32(t_lane + T_S + c * 32, sv);
         tmem_ld32(t_lane + T_DP + c * 32, dv);
@@ -249,8 +258,8 @@ __global__ void __launch_bounds__(192, 1)
           pp[e >> 1] = bpack2<BF16>(pe[0], pe[1]);
           pd[e >> 1] = bpack2<BF16>(de[0], de[1]);
         }
-        tmem_st16(t_lane + T_S + c * 16, pp);
-        tmem_st16(t_lane + T_DP + c * 16, pd);
+        tmem_st16(t_lane + T_S + 64 * wg + cc * 16, pp);
+        tmem_st16(t_lane + T_DP + 64 * wg + cc * 16, pd);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -266,36 +275,33 @@ __global__ void __launch_bounds__(192, 1)
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const bool any = n_iter > 0;
       const size_t o = (static_cast<size_t>(k0 + key) * p.hkv + g) * D;
+      // group 0 writes dV, group 1 writes scale * dK
+      const uint32_t src = wg == 0 ? T_DV : T_DK;
+      const float mul = wg == 0 ? 1.f : p.scale;
+      OutT* dst = reinterpret_cast<OutT*>(wg == 0 ? p.dv : p.dk) + o;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[32], b[32];
-        tmem_ld32(t_lane + T_DV + c * 32, a);
-        tmem_ld32(t_lane + T_DK + c * 32, b);
+        uint32_t a[32];
+        tmem_ld32(t_lane + src + c * 32, a);
         tmem_wait_ld();
         if (key < lk) {
-          uint32_t pa[16], pb[16];
+          uint32_t pa[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            pa[u] = any ? bpack2<BF16>(__uint_as_float(a[2 * u]), __uint_as_float(a[2 * u + 1]))
+          for (int u = 0; u < 16; ++u)
+            pa[u] = any ? bpack2<BF16>(__uint_as_float(a[2 * u]) * mul,
+                                       __uint_as_float(a[2 * u + 1]) * mul)
                         : 0u;
-            pb[u] = any ? bpack2<BF16>(__uint_as_float(b[2 * u]) * p.scale,
-                                       __uint_as_float(b[2 * u + 1]) * p.scale)
-                        : 0u;
-          }
-          uint4* dvp = reinterpret_cast<uint4*>(reinterpret_cast<OutT*>(p.dv) + o + c * 32);
-          uint4* dkp = reinterpret_cast<uint4*>(reinterpret_cast<OutT*>(p.dk) + o + c * 32);
+          uint4* dp4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            dvp[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
-            dkp[u] = make_uint4(pb[4 * u], pb[4 * u + 1], pb[4 * u + 2], pb[4 * u + 3]);
-          }
+          for (int u = 0; u < 4; ++u)
+            dp4[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
         }
       }
     }
   }
   tc_fence_before();
   asm volatile("bar.sync 0;" ::: "memory");
-  if (warp == 4) {
+  if (warp == 8) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(192, 1)
 
 // -------------------------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     mea_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_do,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -351,13 +357,13 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(TBAR(B_KE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
-    mbar_init(TBAR(B_PF), 128);
+    mbar_init(TBAR(B_PF), 256);
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
 
-  if (warp == 5) {
+  if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t loaded = 0;
@@ -397,7 +403,7 @@ __global__ void __launch_bounds__(192, 1)
       for (uint32_t jt = (loaded > 2 ? loaded - 2 : 0); jt < loaded; ++jt)
         mbar_wait(TBAR(B_KF + (jt & 1)), (jt >> 1) & 1, &never, tmo, ecode | 15);
     }
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
       constexpr uint32_t ID_KK = umma_idesc_f16(BF16, 128, 128, false, false);
@@ -419,7 +425,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t ks = sb + C::SMEM_RING + ((jt - 1) & 1) * 2 * C::TILE_BYTES;
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16)
-            mma_ts(tmem + T_DQ, tmem + T_S + k16 * 8,
+            mma_ts(tmem + T_DQ, tmem + T_S + C::packed_col(k16),
                    umma_desc_sw128(ks + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
                    (jt - 1 > 0 || k16 > 0) ? 1u : 0u);
           mma_commit(TBAR(B_KE + ((jt - 1) & 1)));
@@ -450,9 +456,10 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ elementwise (thread = row)
-    const int rl = threadIdx.x;
+    const int wg = threadIdx.x >> 7;                    // column half of this warpgroup
+    const int rl = threadIdx.x & 127;
     const int row = row0 + rl;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const size_t li = static_cast<size_t>(h) * p.total_q + q0 + row;
     const float lse2 = row < lq ? __ldg(p.lse + li) * LOG2E : 0.f;
     const float dl = row < lq ? p.delta[li] : 0.f;
@@ -465,7 +472,8 @@ __global__ void __launch_bounds__(192, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * wg + cc;
         uint32_t sv[32], dv[32];
         tmem_ld32(t_lane + T_S + c * 32, sv);
         tmem_ld32(t_lane + T_DP + c * 32, dv);
@@ -485,7 +493,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           pd[e >> 1] = bpack2<BF16>(de[0], de[1]);
         }
-        tmem_st16(t_lane + T_S + c * 16, pd);
+        tmem_st16(t_lane + T_S + 64 * wg + cc * 16, pd);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -500,8 +508,9 @@ __global__ void __launch_bounds__(192, 1)
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const bool any = n_jt > 0;
       const size_t o = (static_cast<size_t>(q0 + row) * p.hq + h) * D;
+      // group w writes columns [w*D/2, (w+1)*D/2) of dQ
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
         uint32_t a[32];
         tmem_ld32(t_lane + T_DQ + c * 32, a);
         tmem_wait_ld();
@@ -522,7 +531,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   asm volatile("bar.sync 0;" ::: "memory");
-  if (warp == 4) {
+  if (warp == 8) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
