@@ -20,10 +20,11 @@
 // tiles the rows see: S = Q K^T, dP = dO V^T, dS (thread = row), dQ += dS K.
 // TMEM: S [0,128), dP [128,256), dQ [256,256+D).
 //
-// Roles (320 threads): two elementwise warpgroups (warps 0-3 and 4-7; thread = TMEM lane; group
-// w handles columns [64w, 64w+64) of the 128-column S/dP tiles and writes its packed P / dS over
-// the first 32 of them, so the groups never touch each other's columns), warp 8 tcgen05 issuer
-// (owns TMEM), warp 9 TMA producer. Every wait is bounded; no named barriers in the role loops.
+// Roles (NWG*128 + 64 threads): NWG elementwise warpgroups (thread = TMEM lane; group w handles
+// the 32-column chunks [128w/NWG, 128(w+1)/NWG) of the S/dP tiles and writes its packed P / dS
+// over the first half of its own columns, so the groups never touch each other's columns), warp
+// 4*NWG the tcgen05 issuer (owns TMEM), warp 4*NWG+1 the TMA producer. Every wait is bounded; no
+// named barriers in the role loops.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -47,11 +48,16 @@ struct BwdTcCfg {
   static constexpr uint32_t SMEM_BAR = SMEM_RING + 4 * TILE_BYTES;
   static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
   static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
-  static constexpr int THREADS = 320;
-  // Column of the packed 16-bit operand for 16-row step k16 of a 128-column tile: group k16/4
-  // wrote rows 64*(k16/4).. at its own columns 64*(k16/4) + [0, 32).
+  static constexpr int NWG = 4;                          // elementwise warpgroups
+  static constexpr int CPW = 4 / NWG;                      // 32-column chunks per group
+  static constexpr int THREADS = NWG * 128 + 64;
+  static constexpr int W_ISSUE = 4 * NWG, W_LOAD = 4 * NWG + 1;
+  // Column of the packed 16-bit operand for 16-row step k16 of a 128-column tile: chunk k16/2
+  // (32 rows) was packed by its group at the start of the chunk's own 32 columns... precisely,
+  // group w packs its chunks contiguously from column 32*CPW*w.
   __device__ static constexpr uint32_t packed_col(int k16) {
-    return static_cast<uint32_t>(64 * (k16 >> 2) + (k16 & 3) * 8);
+    return static_cast<uint32_t>(32 * CPW * ((k16 >> 1) / CPW) + ((k16 >> 1) % CPW) * 16 +
+                                 (k16 & 1) * 8);
   }
   static constexpr uint32_t TMEM_COLS = 512;
 };
@@ -63,7 +69,7 @@ __device__ __forceinline__ uint32_t bpack2(float lo, float hi) {
 
 // -------------------------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     mea_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_do,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -104,13 +110,13 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(TBAR(B_QE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
-    mbar_init(TBAR(B_PF), 256);
+    mbar_init(TBAR(B_PF), 128 * C::NWG);
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == C::W_ISSUE) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -120,7 +126,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
 
-  if (warp == 9) {
+  if (warp == C::W_LOAD) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t loaded = 0;
@@ -154,7 +160,7 @@ __global__ void __launch_bounds__(320, 1)
       for (uint32_t it = (loaded > 2 ? loaded - 2 : 0); it < loaded; ++it)
         mbar_wait(TBAR(B_QF + (it & 1)), (it >> 1) & 1, &never, tmo, ecode | 15);
     }
-  } else if (warp == 8) {
+  } else if (warp == C::W_ISSUE) {
     // ------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
       constexpr uint32_t ID_KK = umma_idesc_f16(BF16, 128, 128, false, false);  // both K-major
@@ -229,8 +235,8 @@ __global__ void __launch_bounds__(320, 1)
       float slope2 = 0.f;
       if constexpr (ALIBI) slope2 = __ldg(p.slopes + h) * LOG2E;
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * wg + cc;            // 32-column chunk of the tile
+      for (int cc = 0; cc < C::CPW; ++cc) {
+        const int c = C::CPW * wg + cc;       // 32-column chunk of the tile
         uint32_t sv[32], dv[32];
         tmem_ld32(t_lane + T_S + c * 32, sv);
         tmem_ld32(t_lane + T_DP + c * 32, dv);
@@ -258,8 +264,8 @@ __global__ void __launch_bounds__(320, 1)
           pp[e >> 1] = bpack2<BF16>(pe[0], pe[1]);
           pd[e >> 1] = bpack2<BF16>(de[0], de[1]);
         }
-        tmem_st16(t_lane + T_S + 64 * wg + cc * 16, pp);
-        tmem_st16(t_lane + T_DP + 64 * wg + cc * 16, pd);
+        tmem_st16(t_lane + T_S + 32 * C::CPW * wg + cc * 16, pp);
+        tmem_st16(t_lane + T_DP + 32 * C::CPW * wg + cc * 16, pd);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -275,12 +281,17 @@ __global__ void __launch_bounds__(320, 1)
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const bool any = n_iter > 0;
       const size_t o = (static_cast<size_t>(k0 + key) * p.hkv + g) * D;
-      // group 0 writes dV, group 1 writes scale * dK
-      const uint32_t src = wg == 0 ? T_DV : T_DK;
-      const float mul = wg == 0 ? 1.f : p.scale;
-      OutT* dst = reinterpret_cast<OutT*>(wg == 0 ? p.dv : p.dk) + o;
+      // the first half of the groups writes dV, the second half scale * dK, each group its
+      // share of the D columns
+      constexpr int HALF = C::NWG / 2 > 0 ? C::NWG / 2 : 1;
+      const bool is_v = C::NWG == 1 ? true : wg < HALF;
+      const int part = C::NWG == 1 ? 0 : wg % HALF;
+      const uint32_t src = is_v ? T_DV : T_DK;
+      const float mul = is_v ? 1.f : p.scale;
+      OutT* dst = reinterpret_cast<OutT*>(is_v ? p.dv : p.dk) + o;
+      constexpr int CH = (D / 32) / HALF;  // 32-column chunks per group
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = part * CH; c < (part + 1) * CH; ++c) {
         uint32_t a[32];
         tmem_ld32(t_lane + src + c * 32, a);
         tmem_wait_ld();
@@ -301,7 +312,7 @@ __global__ void __launch_bounds__(320, 1)
   }
   tc_fence_before();
   asm volatile("bar.sync 0;" ::: "memory");
-  if (warp == 8) {
+  if (warp == C::W_ISSUE) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
@@ -311,7 +322,7 @@ __global__ void __launch_bounds__(320, 1)
 
 // -------------------------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     mea_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_do,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -357,13 +368,13 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(TBAR(B_KE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
-    mbar_init(TBAR(B_PF), 256);
+    mbar_init(TBAR(B_PF), 128 * C::NWG);
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == C::W_ISSUE) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -373,7 +384,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
 
-  if (warp == 9) {
+  if (warp == C::W_LOAD) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t loaded = 0;
@@ -403,7 +414,7 @@ __global__ void __launch_bounds__(320, 1)
       for (uint32_t jt = (loaded > 2 ? loaded - 2 : 0); jt < loaded; ++jt)
         mbar_wait(TBAR(B_KF + (jt & 1)), (jt >> 1) & 1, &never, tmo, ecode | 15);
     }
-  } else if (warp == 8) {
+  } else if (warp == C::W_ISSUE) {
     // ------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
       constexpr uint32_t ID_KK = umma_idesc_f16(BF16, 128, 128, false, false);
@@ -472,8 +483,8 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * wg + cc;
+      for (int cc = 0; cc < C::CPW; ++cc) {
+        const int c = C::CPW * wg + cc;
         uint32_t sv[32], dv[32];
         tmem_ld32(t_lane + T_S + c * 32, sv);
         tmem_ld32(t_lane + T_DP + c * 32, dv);
@@ -493,7 +504,7 @@ __global__ void __launch_bounds__(320, 1)
           }
           pd[e >> 1] = bpack2<BF16>(de[0], de[1]);
         }
-        tmem_st16(t_lane + T_S + 64 * wg + cc * 16, pd);
+        tmem_st16(t_lane + T_S + 32 * C::CPW * wg + cc * 16, pd);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -508,9 +519,10 @@ __global__ void __launch_bounds__(320, 1)
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const bool any = n_jt > 0;
       const size_t o = (static_cast<size_t>(q0 + row) * p.hq + h) * D;
-      // group w writes columns [w*D/2, (w+1)*D/2) of dQ
+      // group w writes its share of the D columns of dQ (groups past D/32 write none)
+      constexpr int CHQ = (D / 32) / C::NWG > 0 ? (D / 32) / C::NWG : 1;
 #pragma unroll 1
-      for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
+      for (int c = wg * CHQ; c < (wg + 1) * CHQ && c < D / 32; ++c) {
         uint32_t a[32];
         tmem_ld32(t_lane + T_DQ + c * 32, a);
         tmem_wait_ld();
@@ -531,7 +543,7 @@ __global__ void __launch_bounds__(320, 1)
   }
   tc_fence_before();
   asm volatile("bar.sync 0;" ::: "memory");
-  if (warp == 8) {
+  if (warp == C::W_ISSUE) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
