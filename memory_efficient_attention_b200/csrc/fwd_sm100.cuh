@@ -79,7 +79,7 @@ struct FwdCfg {
   // give theirs down to REGS_OTHER so that the two softmax warpgroups can take REGS_SOFTMAX.
   // 256 * REGS_SOFTMAX + 128 * REGS_OTHER must not exceed 64512.
   static constexpr int REGS_SOFTMAX = 216;
-  static constexpr int REGS_OTHER = 64;
+  static constexpr int REGS_OTHER = 72;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_O = 256;                 // O_h at TM_O + h*D
 };
