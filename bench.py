@@ -208,6 +208,20 @@ def aggregate_throughput(units_per_rank: float, world: int, ms_max_over_ranks: f
     return world * units_per_rank / (ms_max_over_ranks * 1e-3)
 
 
+def step_config(args, world):
+    """The `config` of the timed step (shared by both arms)."""
+    from mea_workloads import workload
+    w2, w4 = workload(2), workload(4)
+    return {"workload": ("packed causal GQA+ALiBi prefill (bf16, 32 q / 8 kv heads, D=128, "
+                         f"{w2.total_q} tokens in {len(w2.seqlens_q)} segments U[64,4096]) + "
+                         "split-KV decode (bf16, 64 requests x 1 token, KV U[512,32768], "
+                         "64 q / 8 kv heads, D=128)"),
+            "prefill_seqlens": w2.seqlens_q,
+            "decode_total_kv_tokens": sum(w4.seqlens_k[:max(1, args.decode_requests)]),
+            "l2": "inputs larger than L2 (q 268 MB; K+V 4.3 GB), no flush",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 def oracle_sample(target_flops: float):
     """Leading segments of the packed workload (all 32 heads) until the useful FLOPs reach the
@@ -258,8 +272,7 @@ def run_reference(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "packed causal GQA+ALiBi prefill, bounded sample per step",
-                   "sample": desc},
+        "config": step_config(args, world),
         "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -594,15 +607,7 @@ def run_ours(args, world, rank, local):
     line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic"}
-    cfg = {"workload": ("packed causal GQA+ALiBi prefill (bf16, 32 q / 8 kv heads, D=128, "
-                        f"{w2.total_q} tokens in {len(w2.seqlens_q)} segments U[64,4096]) + "
-                        "split-KV decode (bf16, 64 requests x 1 token, KV U[512,32768], "
-                        "64 q / 8 kv heads, D=128)"),
-           "prefill_seqlens": w2.seqlens_q,
-           "decode_total_kv_tokens": sum(w4.seqlens_k[:max(1, args.decode_requests)]),
-           "l2": "inputs larger than L2 (q 268 MB; K+V 4.3 GB), no flush",
-           "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
-    line["config"] = cfg
+    line["config"] = step_config(args, world)
     if do_fwd:
         fwd_tf = flops / (fwd_ms * 1e-3) / 1e12
         line.update({"value": aggregate_throughput(flops, world, fwd_ms) / 1e12,
