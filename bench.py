@@ -509,7 +509,8 @@ def run_ours(args, world, rank, local):
                    "value": aggregate_throughput(flops, world, f8ms) / 1e12, "unit": "TFLOP/s",
                    "ms_per_call": f8ms, "dtype": "e4m3 in, bf16 out",
                    "roofline": {"bound": "tensor", "achieved": f8tf, "peak": peak8,
-                                "unit": "TFLOP/s", "frac": f8tf / peak8, "traffic": None,
+                                "unit": "TFLOP/s", "frac": f8tf / peak8,
+                                "traffic": traffic_for("mea_fwd_sm100_kernel_e4m3"),
                                 "peak_kind": "dense fp8 = measured bf16 burst x 2 (nominal "
                                              f"4.5 / 2.25 PFLOP/s), {peak_src}",
                                 "kernel": "mea_fwd_sm100_kernel<…, e4m3>"}}
