@@ -468,11 +468,16 @@ __global__ void __launch_bounds__(160, 1)
 // Merge kernel: one CTA per (request, KV group); lse = ln sum_c exp(lse_c),
 // out = sum_c exp(lse_c - lse) O_c, cast to the output dtype.
 template <int D, bool BF16>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     mea_lse_merge_kernel(const DecParams p) {
+  // One CTA per (request b, KV group g): the R heads of the group, all their chunk partials.
+  //   warp w (heads w, w+8, ...): M = max_c lse_c, z = sum_c exp(lse_c - M) -> shared memory;
+  //   then thread (head, 4 columns): O = sum_c exp(lse_c - M) O_c / z with float4 loads.
   const int b = blockIdx.x;
   const int g = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int s_start;
+  __shared__ float s_m[64], s_z[64];
   const int L = __ldg(p.cu_k + b + 1) - __ldg(p.cu_k + b);
   const int n = (L + p.chunk - 1) / p.chunk;
   if (threadIdx.x < 32) {
@@ -483,28 +488,58 @@ __global__ void __launch_bounds__(128)
   const int c0 = s_start;
   using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   OutT* out = reinterpret_cast<OutT*>(p.out);
-  for (int idx = threadIdx.x; idx < p.R * D; idx += blockDim.x) {
-    const int r = idx / D, d = idx - r * D;
-    const int head = g * p.R + r;
-    float M = -INFINITY;
-    for (int c = 0; c < n; ++c)
-      M = fmaxf(M, p.ws_lse[static_cast<size_t>(c0 + c) * p.hq + head]);
-    float z = 0.f, acc = 0.f;
-    if (M != -INFINITY) {
-      for (int c = 0; c < n; ++c) {
-        const size_t slot = static_cast<size_t>(c0 + c) * p.hq + head;
-        const float w = __expf(p.ws_lse[slot] - M);
-        z += w;
-        acc += w * p.ws_o[slot * D + d];
+  constexpr int D4 = D / 4;
+  for (int rb = 0; rb < p.R; rb += 64) {  // heads of the group, 64 at a time
+    const int rn = min(64, p.R - rb);
+    for (int rr = warp; rr < rn; rr += 8) {
+      const int head = g * p.R + rb + rr;
+      float m = -INFINITY;
+      for (int c = lane; c < n; c += 32)
+        m = fmaxf(m, p.ws_lse[static_cast<size_t>(c0 + c) * p.hq + head]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      float z = 0.f;
+      if (m != -INFINITY)
+        for (int c = lane; c < n; c += 32)
+          z += __expf(p.ws_lse[static_cast<size_t>(c0 + c) * p.hq + head] - m);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+      if (lane == 0) {
+        s_m[rr] = m;
+        s_z[rr] = z;
       }
     }
-    const float val = z > 0.f ? acc / z : 0.f;
-    if constexpr (BF16)
-      out[(static_cast<size_t>(b) * p.hq + head) * D + d] = __float2bfloat16_rn(val);
-    else
-      out[(static_cast<size_t>(b) * p.hq + head) * D + d] = __float2half_rn(val);
-    if (d == 0 && p.lse)
-      p.lse[static_cast<size_t>(head) * p.n_seqs + b] = z > 0.f ? M + __logf(z) : -INFINITY;
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < rn * D4; idx += blockDim.x) {
+      const int rr = idx / D4, d = (idx - rr * D4) * 4;
+      const int head = g * p.R + rb + rr;
+      const float m = s_m[rr], z = s_z[rr];
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (m != -INFINITY) {
+#pragma unroll 4
+        for (int c = 0; c < n; ++c) {
+          const size_t slot = static_cast<size_t>(c0 + c) * p.hq + head;
+          const float w = __expf(p.ws_lse[slot] - m);
+          const float4 o = *reinterpret_cast<const float4*>(p.ws_o + slot * D + d);
+          acc.x = fmaf(w, o.x, acc.x);
+          acc.y = fmaf(w, o.y, acc.y);
+          acc.z = fmaf(w, o.z, acc.z);
+          acc.w = fmaf(w, o.w, acc.w);
+        }
+      }
+      const float inv = z > 0.f ? 1.f / z : 0.f;
+      OutT* dst = out + (static_cast<size_t>(b) * p.hq + head) * D + d;
+      if constexpr (BF16) {
+        reinterpret_cast<__nv_bfloat162*>(dst)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        reinterpret_cast<__nv_bfloat162*>(dst)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      } else {
+        reinterpret_cast<__half2*>(dst)[0] = __floats2half2_rn(acc.x * inv, acc.y * inv);
+        reinterpret_cast<__half2*>(dst)[1] = __floats2half2_rn(acc.z * inv, acc.w * inv);
+      }
+      if (d == 0 && p.lse)
+        p.lse[static_cast<size_t>(head) * p.n_seqs + b] = z > 0.f ? m + __logf(z) : -INFINITY;
+    }
+    __syncthreads();
   }
 }
 

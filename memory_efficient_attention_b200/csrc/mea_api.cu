@@ -207,7 +207,7 @@ int launch_dec_t(const CUtensorMap& tk, const CUtensorMap& tv, const mea::DecPar
   if (grid > 0) kern<<<grid, mea::DecCfg<D>::THREADS, smem, stream>>>(tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return MEA_ERR_CUDA;
   dim3 mgrid(p.n_seqs, n_kv_heads);
-  mea::mea_lse_merge_kernel<D, BF16><<<mgrid, 128, 0, stream>>>(p);
+  mea::mea_lse_merge_kernel<D, BF16><<<mgrid, 256, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
 
