@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       mbar_init(TBAR(B_QE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
-    mbar_init(TBAR(B_PF), 128 * C::NWG);
+    mbar_init(TBAR(B_PF), 4 * C::NWG);  // one elected arrival per elementwise warp
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
     *abort_flag = 0;
@@ -269,7 +269,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(TBAR(B_PF));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(TBAR(B_PF));
     }
     // ---- epilogue: dV, scale * dK for this thread's key
     if (ok) {
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       mbar_init(TBAR(B_KE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
-    mbar_init(TBAR(B_PF), 128 * C::NWG);
+    mbar_init(TBAR(B_PF), 4 * C::NWG);  // one elected arrival per elementwise warp
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
     *abort_flag = 0;
@@ -508,7 +509,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(TBAR(B_PF));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(TBAR(B_PF));
     }
     if (ok) {
       ok = mbar_wait(TBAR(B_ACC), 0, abort_flag, tmo, ecode | 6);

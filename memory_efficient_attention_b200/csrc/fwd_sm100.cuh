@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(BAR(B_SF + h), 1);
-      mbar_init(BAR(B_PF + h), 128);
+      mbar_init(BAR(B_PF + h), 4);  // one elected arrival per softmax warp
       mbar_init(BAR(B_OF + h), 1);
       mbar_init(BAR(B_OE + h), 128);
     }
@@ -594,9 +594,11 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st32(t_o + c4 * 32, o);
           }
         }
+        // Each thread's P stores complete, then one lane per warp publishes the warp's rows.
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(B_PF + h));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_PF + h));
         ++tile;
       }
       if (!ok) break;
