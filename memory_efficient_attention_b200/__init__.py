@@ -336,7 +336,8 @@ class LowerTriangularMask:
 
 def memory_efficient_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                attn_bias=None, scale: Optional[float] = None) -> torch.Tensor:
-    """Exact attention on BMHK ``[B, M, H, K]`` or BMGHK ``[B, M, G, Hq, K]`` tensors.
+    """Exact attention on BMHK ``[B, M, H, K]`` or BMGHK ``[B, M, G, Hq, K]`` tensors;
+    differentiable (the backward runs mea_backward) when an input requires grad.
 
     BMGHK: k/v are ``[B, Mk, G, 1, K]`` (one KV head per group, shared by the group's Hq query
     heads) and the output is ``[B, M, G, Hq, K]``. With a block-diagonal mask B must be 1 and the
@@ -378,9 +379,35 @@ def _bmhk_packed(qp, kp, vp, b, m, mk, attn_bias, scale):
         causal = isinstance(attn_bias, LowerTriangularMask)
         if attn_bias is not None and not isinstance(attn_bias, LowerTriangularMask):
             raise MeaError(_lib.MEA_ERR_MASK, f"unsupported attn_bias {type(attn_bias).__name__}")
+    max_k = max(attn_bias.kv_seqlen) if isinstance(attn_bias, BlockDiagonalMask) and \
+        attn_bias.kv_seqlen else mk
+    if torch.is_grad_enabled() and (qp.requires_grad or kp.requires_grad or vp.requires_grad):
+        return _PackedAttention.apply(qp, kp, vp, cu_q, cu_k, max_q, max_k, causal, slopes, scale)
     out, _ = attention_packed(qp, kp, vp, cu_q, cu_k, max_q, causal=causal, alibi_slopes=slopes,
                               scale=scale, return_lse=False)
     return out
+
+
+class _PackedAttention(torch.autograd.Function):
+    """Packed attention with its gradients: forward through mea_forward (keeping out and lse),
+    backward through mea_backward."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, causal, slopes, scale):
+        out, lse = attention_packed(q, k, v, cu_q, cu_k, max_q, causal=causal,
+                                    alibi_slopes=slopes, scale=scale)
+        ctx.save_for_backward(q, k, v, out, lse, cu_q, cu_k)
+        ctx.args = (max_q, max_k, causal, slopes, scale)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse, cu_q, cu_k = ctx.saved_tensors
+        max_q, max_k, causal, slopes, scale = ctx.args
+        dq, dk, dv = attention_packed_backward(q, k, v, out, lse, dout.contiguous(), cu_q, cu_k,
+                                               max_q, max_k, causal=causal, alibi_slopes=slopes,
+                                               scale=scale)
+        return dq, dk, dv, None, None, None, None, None, None, None
 
 
 def device_error(clear: bool = True) -> int:
