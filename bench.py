@@ -47,6 +47,8 @@ def parse():
                     help="skip the paged-cache decode measurement")
     ap.add_argument("--no-fp8", dest="fp8", action="store_false",
                     help="skip the FP8 forward measurement")
+    ap.add_argument("--no-long", dest="long", action="store_false",
+                    help="skip the long-context (16384-token) prefill measurement")
     ap.add_argument("--paged-block-size", type=int, default=16,
                     help="slots per cache block of the paged decode measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -515,6 +517,49 @@ def run_ours(args, world, rank, local):
                                              f"4.5 / 2.25 PFLOP/s), {peak_src}",
                                 "kernel": "mea_fwd_sm100_kernel<…, e4m3>"}}
 
+    # ---- long-context causal prefill (16384 tokens, GQA 64/8, no ALiBi), timed on its own
+    long_obj = None
+    if do_fwd and args.long:
+        w3 = workload(3)
+        g.manual_seed(w3.seed)
+        t3 = w3.seqlens_q[0]
+        q3 = torch.randn((t3, 64, 128), generator=g, device=dev, dtype=torch.float32).bfloat16()
+        k3 = torch.randn((t3, 8, 128), generator=g, device=dev, dtype=torch.float32).bfloat16()
+        v3 = torch.randn((t3, 8, 128), generator=g, device=dev, dtype=torch.float32).bfloat16()
+        cu3 = cu_seqlens(w3.seqlens_q).to(dev)
+        out3 = torch.empty_like(q3)
+        lse3 = torch.empty((64, t3), dtype=torch.float32, device=dev)
+        flops3 = fwd_flops(w3.seqlens_q, 64, 128)
+
+        def fwd3():
+            mea.attention_packed(q3, k3, v3, cu3, cu3, t3, causal=True, scale=w3.scale,
+                                 out=out3, lse=lse3)
+        for _ in range(args.warmup):
+            fwd3()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fwd3()
+        b.record(stream)
+        barrier(world)
+        l3ms = dist_max(a.elapsed_time(b), world) / args.steps
+        code = mea.device_error()
+        if code:
+            raise RuntimeError(f"device error word {code:#x} during the long prefill")
+        l3tf = flops3 / (l3ms * 1e-3) / 1e12
+        peak3 = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        long_obj = {"metric": "attention fwd TFLOP/s (causal prefill, 16384 tokens, GQA 64/8, "
+                              "D=128, bf16)",
+                    "value": aggregate_throughput(flops3, world, l3ms) / 1e12,
+                    "unit": "TFLOP/s", "ms_per_call": l3ms,
+                    "roofline": {"bound": "tensor", "achieved": l3tf, "peak": peak3,
+                                 "unit": "TFLOP/s", "frac": l3tf / peak3, "traffic": None,
+                                 "peak_kind": f"dense bf16 burst, {peak_src}",
+                                 "kernel": "mea_fwd_sm100_kernel<128, bf16, causal>",
+                                 "flops_per_launch": flops3}}
+        del q3, k3, v3, out3, lse3
+
     # ---- paged-cache decode of the same requests, timed on its own (not part of the step)
     paged_obj = None
     if do_dec and args.paged:
@@ -638,6 +683,8 @@ def run_ours(args, world, rank, local):
                          "roofline": dec_obj["roofline"]})
     if fp8_obj is not None:
         line["fp8_forward"] = fp8_obj
+    if long_obj is not None:
+        line["long_prefill"] = long_obj
     if paged_obj is not None:
         line["paged_decode"] = paged_obj
     if bwd_obj is not None:

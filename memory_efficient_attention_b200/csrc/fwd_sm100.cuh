@@ -50,6 +50,15 @@ struct FwdParams {
   int tok_per_tile;  // 128 / P tokens per sub-tile
   int t_max;         // max sub-tile pairs of a segment
   long long n_items; // t_max * n_seqs * n_hb
+  // Division-free scheduling (an integer division runs partly on the MUFU, which the softmax
+  // keeps saturated): P and 2 * tok_per_tile are powers of two; the KV group of head block hb
+  // is (hb * g_mul) >> 32 with g_mul = ceil(2^32 / (R / P)) (exact for hb * (R / P) < 2^32);
+  // a CTA advances through the items by gridDim.x = step_tr * (n_seqs * n_hb) +
+  // step_seg * n_hb + step_hb.
+  int log2_p;
+  int log2_tpp;
+  unsigned long long g_mul;
+  int step_tr, step_seg, step_hb;
   float c1;          // scale * log2(e) (times the q and k descales for 8-bit inputs)
   float o_scale;     // multiplies O before the division by l (the v descale; 1 for 16-bit)
   unsigned long long timeout_ns;
@@ -71,15 +80,20 @@ struct FwdCfg {
   static constexpr uint32_t SMEM_Q = 0;                 // two Q sub-tiles
   static constexpr uint32_t SMEM_KV = 2 * TILE_BYTES;
   static constexpr uint32_t SMEM_BAR = SMEM_KV + NS * TILE_BYTES;
-  static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 512 + 1024;
+  // cu_seqlens_q / cu_seqlens_k copied to shared memory when they have at most SEQ_CACHE
+  // entries: every role decodes every work item, including the empty ones it skips, and a
+  // global-memory round trip per skipped item stalls each item boundary.
+  static constexpr int SEQ_CACHE = 192;
+  static constexpr uint32_t SMEM_SEQ = SMEM_BAR + 512;
+  static constexpr uint32_t SMEM_TOTAL = SMEM_SEQ + 2 * SEQ_CACHE * 4 + 1024;
   static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
   static_assert(!E8 || D == 128, "8-bit inputs: D = 128 (one 128-byte swizzle atom per row)");
   static constexpr int THREADS = 384;
   // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); warps 8-11
   // give theirs down to REGS_OTHER so that the two softmax warpgroups can take REGS_SOFTMAX.
   // 256 * REGS_SOFTMAX + 128 * REGS_OTHER must not exceed 64512.
-  static constexpr int REGS_SOFTMAX = 216;
-  static constexpr int REGS_OTHER = 72;
+  static constexpr int REGS_SOFTMAX = E8 ? 216 : 208;
+  static constexpr int REGS_OTHER = E8 ? 72 : 80;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_O = 256;                 // O_h at TM_O + h*D
 };
@@ -90,23 +104,75 @@ struct FwdItem {
   bool live;
 };
 
-__device__ __forceinline__ FwdItem fwd_decode_item(const FwdParams& p, long long lin,
-                                                   bool causal) {
-  FwdItem it;
+__device__ __forceinline__ int lds_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// Position of a CTA in the item list: item tr * (n_seqs * n_hb) + seg * n_hb + hb.
+struct FwdIter {
+  int tr, seg, hb;
+};
+
+// The CTA's first item (the only divisions of the schedule; item blockIdx.x exists because
+// the grid is never larger than the item count).
+__device__ __forceinline__ FwdIter fwd_iter_first(const FwdParams& p) {
+  FwdIter s;
   const long long per = static_cast<long long>(p.n_seqs) * p.n_hb;
-  const int tr = static_cast<int>(lin / per);
-  const int rem = static_cast<int>(lin - static_cast<long long>(tr) * per);
-  it.seg = rem / p.n_hb;
-  it.hb = rem - it.seg * p.n_hb;
-  it.q0 = __ldg(p.cu_q + it.seg);
-  it.lq = __ldg(p.cu_q + it.seg + 1) - it.q0;
-  it.k0 = __ldg(p.cu_k + it.seg);
-  it.lk = __ldg(p.cu_k + it.seg + 1) - it.k0;
-  const int tpp = 2 * p.tok_per_tile;
-  const int np = (it.lq + tpp - 1) / tpp;
+  const long long b = blockIdx.x;
+  s.tr = static_cast<int>(b / per);
+  const int rem = static_cast<int>(b - static_cast<long long>(s.tr) * per);
+  s.seg = rem / p.n_hb;
+  s.hb = rem - s.seg * p.n_hb;
+  return s;
+}
+
+// Item + gridDim.x: each mixed-radix digit carries at most once (step_hb < n_hb,
+// step_seg < n_seqs). The list ends when tr reaches t_max.
+__device__ __forceinline__ void fwd_iter_next(FwdIter& s, const FwdParams& p) {
+  s.hb += p.step_hb;
+  s.seg += p.step_seg;
+  s.tr += p.step_tr;
+  if (s.hb >= p.n_hb) {
+    s.hb -= p.n_hb;
+    ++s.seg;
+  }
+  if (s.seg >= p.n_seqs) {
+    s.seg -= p.n_seqs;
+    ++s.tr;
+  }
+}
+
+__device__ __forceinline__ int fwd_group_of(const FwdParams& p, int hb) {
+  return static_cast<int>((static_cast<unsigned long long>(hb) * p.g_mul) >> 32);
+}
+
+// s_cu: shared-memory address of the cached cu_seqlens_q (cu_seqlens_k follows SEQ_CACHE
+// entries later), or 0 when they are read from global memory.
+template <int SEQ_CACHE>
+__device__ __forceinline__ FwdItem fwd_decode_item(const FwdParams& p, const FwdIter& s,
+                                                   bool causal, uint32_t s_cu) {
+  FwdItem it;
+  const int tr = s.tr;
+  it.seg = s.seg;
+  it.hb = s.hb;
+  if (s_cu != 0) {
+    const uint32_t a = s_cu + 4u * static_cast<uint32_t>(it.seg);
+    it.q0 = lds_s32(a);
+    it.lq = lds_s32(a + 4) - it.q0;
+    it.k0 = lds_s32(a + 4 * SEQ_CACHE);
+    it.lk = lds_s32(a + 4 * SEQ_CACHE + 4) - it.k0;
+  } else {
+    it.q0 = __ldg(p.cu_q + it.seg);
+    it.lq = __ldg(p.cu_q + it.seg + 1) - it.q0;
+    it.k0 = __ldg(p.cu_k + it.seg);
+    it.lk = __ldg(p.cu_k + it.seg + 1) - it.k0;
+  }
+  const int np = (it.lq + (1 << p.log2_tpp) - 1) >> p.log2_tpp;
   const int t = causal ? (p.t_max - 1 - tr) : tr;
   it.live = (t >= 0) && (t < np);
-  it.tok0 = t * tpp;
+  it.tok0 = t << p.log2_tpp;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int first = it.tok0 + h * p.tok_per_tile;
@@ -303,6 +369,15 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  int32_t* s_cu = reinterpret_cast<int32_t*>(smem + C::SMEM_SEQ);
+  const bool seq_cached = p.n_seqs + 1 <= C::SEQ_CACHE;
+  if (seq_cached) {
+    for (int i = threadIdx.x; i <= p.n_seqs; i += blockDim.x) {
+      s_cu[i] = __ldg(p.cu_q + i);
+      s_cu[C::SEQ_CACHE + i] = __ldg(p.cu_k + i);
+    }
+  }
+  const uint32_t s_cu_addr = seq_cached ? sbase + C::SMEM_SEQ : 0u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -316,11 +391,11 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       uint32_t kv_cnt = 0, q_cnt = 0;
       bool ok = true;
-      for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
-        const FwdItem it = fwd_decode_item(p, lin, CAUSAL);
+      for (FwdIter cur = fwd_iter_first(p); cur.tr < p.t_max && ok; fwd_iter_next(cur, p)) {
+        const FwdItem it = fwd_decode_item<C::SEQ_CACHE>(p, cur, CAUSAL, s_cu_addr);
         const int nmax = max(it.n_kv[0], it.n_kv[1]);
         if (!it.live || nmax == 0) continue;
-        const int g = (it.hb * p.P) / p.R;
+        const int g = fwd_group_of(p, it.hb);
         ok = mbar_wait(BAR(B_QE), (q_cnt & 1u) ^ 1u, abort_flag, tmo, ecode | 1);
         if (!ok) break;
         mbar_arrive_expect_tx(BAR(B_QF), 2 * C::TILE_BYTES);
@@ -330,7 +405,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int a = 0; a < C::ATOMS; ++a)
             tma_load_3d(q_s + h * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_q, BAR(B_QF),
                         a * C::ATOM_COLS,
-                        it.hb * p.P, it.q0 + it.tok0 + h * p.tok_per_tile);
+                        it.hb << p.log2_p, it.q0 + it.tok0 + h * p.tok_per_tile);
         ++q_cnt;
         for (int j = 0; j < nmax && ok; ++j) {
 #pragma unroll 1
@@ -348,6 +423,28 @@ __global__ void __launch_bounds__(384, 1)
                           it.k0 + (nmax - 1 - j) * 128);
             ++kv_cnt;
           }
+        }
+        // Warm L2 with the next item's Q tiles and its first two K/V tiles while this item's
+        // last steps are still being computed: the next Q can only be loaded once this item's
+        // last Q K^T has finished, and fetched cold from HBM it would stall the item boundary.
+        FwdIter nx = cur;
+        for (fwd_iter_next(nx, p); ok && nx.tr < p.t_max; fwd_iter_next(nx, p)) {
+          const FwdItem nt = fwd_decode_item<C::SEQ_CACHE>(p, nx, CAUSAL, s_cu_addr);
+          const int nm = max(nt.n_kv[0], nt.n_kv[1]);
+          if (!nt.live || nm == 0) continue;
+          const int ng = fwd_group_of(p, nt.hb);
+#pragma unroll
+          for (int a = 0; a < C::ATOMS; ++a) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tma_prefetch_l2_3d(&tm_q, a * C::ATOM_COLS, nt.hb << p.log2_p,
+                                 nt.q0 + nt.tok0 + h * p.tok_per_tile);
+            for (int j = 0; j < min(nm, 2); ++j) {
+              tma_prefetch_l2_3d(&tm_k, a * C::ATOM_COLS, ng, nt.k0 + (nm - 1 - j) * 128);
+              tma_prefetch_l2_3d(&tm_v, a * C::ATOM_COLS, ng, nt.k0 + (nm - 1 - j) * 128);
+            }
+          }
+          break;
         }
       }
       if (!ok) {
@@ -373,8 +470,8 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t kv_cnt = 0, q_cnt = 0;
       uint32_t pv_cnt[2] = {0, 0}, oe_cnt[2] = {0, 0};
       bool ok = true;
-      for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
-        const FwdItem it = fwd_decode_item(p, lin, CAUSAL);
+      for (FwdIter cur = fwd_iter_first(p); cur.tr < p.t_max && ok; fwd_iter_next(cur, p)) {
+        const FwdItem it = fwd_decode_item<C::SEQ_CACHE>(p, cur, CAUSAL, s_cu_addr);
         const int nmax = max(it.n_kv[0], it.n_kv[1]);
         if (!it.live || nmax == 0) continue;
         ok = mbar_wait(BAR(B_QF), q_cnt & 1u, abort_flag, tmo, ecode | 6);
@@ -467,12 +564,13 @@ __global__ void __launch_bounds__(384, 1)
     constexpr float LN2 = 0.6931471805599453f;
     uint32_t tile = 0, ocnt = 0;
     bool ok = true;
-    for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
-      const FwdItem it = fwd_decode_item(p, lin, CAUSAL);
+    const bool out_al32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
+    for (FwdIter cur = fwd_iter_first(p); cur.tr < p.t_max && ok; fwd_iter_next(cur, p)) {
+      const FwdItem it = fwd_decode_item<C::SEQ_CACHE>(p, cur, CAUSAL, s_cu_addr);
       if (!it.live) continue;
       const int sub0 = it.tok0 + h * p.tok_per_tile;  // first token of this sub-tile
-      const int tok = sub0 + r / p.P;
-      const int head = it.hb * p.P + (r % p.P);
+      const int tok = sub0 + (r >> p.log2_p);
+      const int head = (it.hb << p.log2_p) + (r & (p.P - 1));
       const bool row_valid = tok < it.lq;
       const int nh = it.n_kv[h];
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
@@ -609,25 +707,32 @@ __global__ void __launch_bounds__(384, 1)
       ++ocnt;
       tc_fence_after();
       const float inv_l = l > 0.f ? p.o_scale / l : 0.f;
-#pragma unroll 1
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        uint32_t o[32];
-        tmem_ld32(t_o + c4 * 32, o);
-        tmem_wait_ld();
-        if (row_valid) {
-          uint32_t pk[16];
+      // The whole O row in one round of loads; once they have landed O_h is free for the next
+      // item's P V, before any of the global stores.
+      uint32_t o[D];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l,
-                                __uint_as_float(o[2 * i + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-        }
-      }
+      for (int c4 = 0; c4 < D / 32; ++c4)
+        tmem_ld32(t_o + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c4 * 32]));
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(BAR(B_OE + h));
+      if (row_valid) {
+#pragma unroll
+        for (int i = 0; i < D / 2; ++i)
+          o[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l,
+                             __uint_as_float(o[2 * i + 1]) * inv_l);
+        // Each thread writes its own row: 32-byte stores fill whole sectors (rows are 128 or
+        // 256 bytes, so they stay 32-byte aligned when out is).
+        if (out_al32) {
+#pragma unroll
+          for (int i = 0; i < D / 16; ++i) st_global_v8(orow + i * 16, &o[8 * i]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i)
+            dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
+      }
       if (row_valid && p.lse)
         p.lse[static_cast<size_t>(head) * p.total_q + it.q0 + tok] =
             l > 0.f ? (m_ref + __log2f(l)) * LN2 : -INFINITY;

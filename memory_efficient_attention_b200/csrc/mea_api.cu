@@ -91,6 +91,30 @@ int largest_pow2_divisor(int x, int cap) {
   return p;
 }
 
+// Constants of the forward kernel's division-free schedule (see FwdParams): shifts for the
+// power-of-two packing factors, the multiplier that maps a head block to its KV group, and the
+// per-CTA stride through the item list in mixed radix (t_max, n_seqs, n_hb).
+// Returns false when (hb * g_mul) >> 32 would not be exact for every head block
+// ((n_hb - 1) * (d - 1) < 2^32 is sufficient).
+static bool fwd_schedule_constants(mea::FwdParams& p, int grid) {
+  int l2p = 0;
+  while ((1 << l2p) < p.P) ++l2p;
+  int l2t = 0;
+  while ((1 << l2t) < 2 * p.tok_per_tile) ++l2t;
+  p.log2_p = l2p;
+  p.log2_tpp = l2t;
+  const unsigned long long d = static_cast<unsigned long long>(p.R / p.P);
+  p.g_mul = ((1ull << 32) + d - 1) / d;
+  if (static_cast<unsigned long long>(p.n_hb - 1) * (d - 1) >= (1ull << 32)) return false;
+  const long long per = static_cast<long long>(p.n_seqs) * p.n_hb;
+  const long long g = grid;
+  p.step_tr = static_cast<int>(g / per);
+  const long long r = g % per;
+  p.step_seg = static_cast<int>(r / p.n_hb);
+  p.step_hb = static_cast<int>(r % p.n_hb);
+  return true;
+}
+
 // ------------------------------------------------------------------------------------------
 // Forward launch dispatch.
 // ------------------------------------------------------------------------------------------
@@ -365,6 +389,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, float* 
       !encode_3d(&tv, v, in_dtype, head_dim, n_heads_kv, tk_rows, box0, 1, 128))
     return MEA_ERR_CUDA;
   const int grid = static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms);
+  if (!fwd_schedule_constants(p, grid)) return MEA_ERR_HEADS;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool causal = mask_kind == MEA_MASK_CAUSAL;
   const bool alibi = alibi_slopes != nullptr;
