@@ -186,6 +186,15 @@ def test_lq_ne_lk_bottom_right_and_empty():
         check_packed(lq, lk, 8, 4, 128, torch.bfloat16, causal, True, 0.09, 77)
 
 
+@pytest.mark.parametrize("n_seqs", [191, 192, 300])
+def test_many_segments(n_seqs):
+    # the forward keeps cu_seqlens in shared memory for up to 191 segments and reads them from
+    # global memory beyond that; both sides of the limit, causal with GQA (R = 3)
+    g = torch.Generator().manual_seed(n_seqs)
+    lens = torch.randint(1, 161, (n_seqs,), generator=g).tolist()
+    check_packed(lens, lens, 6, 2, 64, torch.float16, True, False, 0.125, 900 + n_seqs)
+
+
 def test_max_seqlen_upper_bound():
     lens = [50, 20]
     check_packed(lens, lens, 4, 2, 64, torch.float16, True, False, 0.125, 5, max_seqlen_q=70)
