@@ -83,6 +83,11 @@ typedef enum {
  *   alibi_slopes  NULL, or DEVICE fp32 [n_heads_q] slopes (2^(-8(h+1)/Hq) is the usual choice).
  *   dtype         mea_dtype of q, k, v and out.
  * Returns MEA_OK or a negative mea_status. Segments with L_q = 0 produce nothing.
+ * MEA_ERR_HEADS also covers head counts so large that the kernel's integer head-block-to-group
+ * mapping could round wrongly ((H/P - 1) * (R/P - 1) >= 2^32, with R = n_heads_q / n_heads_kv
+ * and P its largest power-of-two divisor up to 128); no realistic head count reaches it.
+ * Performance: cu_seqlens_q/k of up to 191 segments are kept in on-chip memory; longer lists
+ * are read from global memory as the work is scheduled.
  */
 int mea_forward(const void* q, const void* k, const void* v, void* out, float* lse,
                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int n_seqs,
