@@ -10,9 +10,16 @@ Public API (names follow the pages' vocabulary):
   ``[B, M, H, K]`` or BMGHK ``[B, M, G, Hq, K]`` tensors, the call of the 7minutos page's packed
   and grouped examples; ``attn_bias`` is a :class:`BlockDiagonalMask`,
   :class:`BlockDiagonalCausalMask` or :class:`LowerTriangularMask`, optionally with ALiBi slopes.
-* :func:`attention_packed` — the raw packed-varlen call ``[T, H, D]`` with ``cu_seqlens``.
-* :func:`decode_splitkv` — one query token per request against a packed KV cache.
+* :func:`attention_packed` — the raw packed-varlen call ``[T, H, D]`` with ``cu_seqlens``;
+  :func:`attention_packed_fp8` the same with e4m3 inputs; :func:`attention_packed_backward` its
+  gradients.
+* :func:`decode_splitkv` — one query token per request against a packed KV cache;
+  :func:`decode_paged` against a block cache; :func:`decode_splitkv_noalloc` without a workspace.
 * :func:`alibi_slopes` — ``2^(-8(h+1)/H)``.
+
+Caller-provided outputs and workspaces must be contiguous tensors of exactly the documented
+shape, dtype and device: the library writes through their pointers with sizes taken from the
+other arguments, so a mismatch raises here instead.
 """
 from __future__ import annotations
 
@@ -27,8 +34,9 @@ from ._lib import MeaError  # noqa: F401
 __all__ = [
     "memory_efficient_attention", "attention_packed", "attention_packed_fp8",
     "attention_packed_backward", "backward_workspace_size", "decode_splitkv", "decode_paged",
-    "decode_splitkv_noalloc", "decode_workspace_size", "wait_selftest", "alibi_slopes", "BlockDiagonalMask", "BlockDiagonalCausalMask",
-    "LowerTriangularMask", "device_error", "set_wait_timeout_ns", "MeaError", "library_path",
+    "decode_splitkv_noalloc", "decode_workspace_size", "wait_selftest", "alibi_slopes",
+    "BlockDiagonalMask", "BlockDiagonalCausalMask", "LowerTriangularMask", "device_error",
+    "set_wait_timeout_ns", "MeaError", "library_path",
 ]
 
 library_path = _lib.LIB_PATH
@@ -48,6 +56,41 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def _stream(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
+
+
+def _on_device(device: torch.device, **tensors) -> None:
+    """Each given tensor (None is skipped) must be a CUDA tensor on ``device``: the kernels
+    dereference every pointer on that GPU."""
+    for name, t in tensors.items():
+        if t is not None and (not t.is_cuda or t.device != device):
+            raise MeaError(_lib.MEA_ERR_DEVICE, f"{name} must be a CUDA tensor on {device}")
+
+
+def _check_buffer(name: str, t: torch.Tensor, shape, dtype: torch.dtype,
+                  device: torch.device) -> torch.Tensor:
+    """A caller-provided output must match exactly (the library writes through its pointer)."""
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != device \
+            or not t.is_contiguous():
+        raise MeaError(_lib.MEA_ERR_SHAPE,
+                       f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} "
+                       f"on {device}")
+    return t
+
+
+def _check_workspace(t: torch.Tensor, device: torch.device) -> int:
+    """A caller-provided workspace: contiguous, on ``device``; returns its size in bytes (the
+    library checks that it is large enough)."""
+    if t.device != device or not t.is_contiguous():
+        raise MeaError(_lib.MEA_ERR_WORKSPACE, f"workspace must be contiguous on {device}")
+    return t.numel() * t.element_size()
+
+
+def _check_cu(name: str, t: torch.Tensor, n: int, device: torch.device) -> torch.Tensor:
+    """cu_seqlens: int32 ``[n]`` on ``device`` (made contiguous)."""
+    if t.dtype != torch.int32 or t.dim() != 1 or t.numel() != n:
+        raise MeaError(_lib.MEA_ERR_SHAPE, f"{name} must be int32 [{n}]")
+    _on_device(device, **{name: t})
+    return t.contiguous()
 
 
 def alibi_slopes(n_heads: int, device=None) -> torch.Tensor:
@@ -79,16 +122,20 @@ def attention_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     tk, hkv, _ = k.shape
     if k.shape != v.shape or k.shape[2] != d or q.dtype != k.dtype or k.dtype != v.dtype:
         raise MeaError(_lib.MEA_ERR_SHAPE, "q/k/v shapes or dtypes disagree")
+    _on_device(q.device, k=k, v=v)
     n_seqs = cu_seqlens_q.numel() - 1
-    if cu_seqlens_k.numel() != n_seqs + 1 or cu_seqlens_q.dtype != torch.int32 \
-            or cu_seqlens_k.dtype != torch.int32:
-        raise MeaError(_lib.MEA_ERR_SHAPE, "cu_seqlens must be int32 [n_seqs+1]")
+    cu_seqlens_q = _check_cu("cu_seqlens_q", cu_seqlens_q, n_seqs + 1, q.device)
+    cu_seqlens_k = _check_cu("cu_seqlens_k", cu_seqlens_k, n_seqs + 1, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
+    else:
+        _check_buffer("out", out, (tq, hq, d), q.dtype, q.device)
     if return_lse and lse is None:
         lse = torch.empty((hq, tq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check_buffer("lse", lse, (hq, tq), torch.float32, q.device)
     if alibi_slopes is not None:
         alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
     rc = _lib.load().mea_forward(
@@ -112,16 +159,25 @@ def attention_packed_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     for t in (q, k, v):
         if not t.is_cuda or t.dtype != torch.float8_e4m3fn:
             raise MeaError(_lib.MEA_ERR_DTYPE, "q, k, v must be float8_e4m3fn on the GPU")
+    if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape or k.shape[2] != q.shape[2]:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "q [T_q, Hq, D], k/v [T_k, Hkv, D]")
+    _on_device(q.device, k=k, v=v)
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
     tq, hq, d = q.shape
     tk, hkv, _ = k.shape
     n_seqs = cu_seqlens_q.numel() - 1
+    cu_seqlens_q = _check_cu("cu_seqlens_q", cu_seqlens_q, n_seqs + 1, q.device)
+    cu_seqlens_k = _check_cu("cu_seqlens_k", cu_seqlens_k, n_seqs + 1, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty((tq, hq, d), dtype=out_dtype, device=q.device)
+    else:
+        _check_buffer("out", out, (tq, hq, d), out.dtype, q.device)
     if lse is None:
         lse = torch.empty((hq, tq), dtype=torch.float32, device=q.device)
+    else:
+        _check_buffer("lse", lse, (hq, tq), torch.float32, q.device)
     if alibi_slopes is not None:
         alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
     rc = _lib.load().mea_forward_fp8(
@@ -153,6 +209,10 @@ def attention_packed_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     for t in (q, k, v, out, dout):
         if not t.is_cuda:
             raise MeaError(_lib.MEA_ERR_DEVICE, "tensors must live on the GPU")
+    _on_device(q.device, k=k, v=v, out=out, lse=lse, dout=dout)
+    if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape or k.shape[2] != q.shape[2] \
+            or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "q [T_q, Hq, D], k/v [T_k, Hkv, D] of one dtype")
     q, k, v, out, dout = (t.contiguous() for t in (q, k, v, out, dout))
     lse = lse.contiguous()
     tq, hq, d = q.shape
@@ -161,6 +221,8 @@ def attention_packed_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             or lse.dtype != torch.float32 or dout.dtype != q.dtype or out.dtype != q.dtype:
         raise MeaError(_lib.MEA_ERR_SHAPE, "out/dout must match q; lse must be fp32 [Hq, T_q]")
     n_seqs = cu_seqlens_q.numel() - 1
+    cu_seqlens_q = _check_cu("cu_seqlens_q", cu_seqlens_q, n_seqs + 1, q.device)
+    cu_seqlens_k = _check_cu("cu_seqlens_k", cu_seqlens_k, n_seqs + 1, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if alibi_slopes is not None:
@@ -168,16 +230,16 @@ def attention_packed_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     need = backward_workspace_size(tq, hq)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = _check_workspace(workspace, q.device)
+    dq = torch.empty_like(q) if dq is None else _check_buffer("dq", dq, q.shape, q.dtype, q.device)
+    dk = torch.empty_like(k) if dk is None else _check_buffer("dk", dk, k.shape, k.dtype, q.device)
+    dv = torch.empty_like(v) if dv is None else _check_buffer("dv", dv, v.shape, v.dtype, q.device)
     rc = _lib.load().mea_backward(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
         _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), n_seqs, tq, tk, int(max_seqlen_q),
         int(max_seqlen_k), hq, hkv, d, float(scale),
         _lib.MEA_MASK_CAUSAL if causal else _lib.MEA_MASK_NONE, _ptr(alibi_slopes),
-        _dtype_code(q.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream(q.device))
+        _dtype_code(q.dtype), _ptr(workspace), ws_bytes, _stream(q.device))
     _lib.check(rc, "mea_backward")
     return dq, dk, dv
 
@@ -195,11 +257,15 @@ def decode_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
                    lse: Optional[torch.Tensor] = None, return_lse: bool = True):
     """Single-token decode: q ``[B, Hq, D]`` against packed k/v ``[T_k, Hkv, D]``.
     Returns ``(out [B, Hq, D], lse [Hq, B] or None)``."""
-    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+    if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape or k.shape[2] != q.shape[2]:
         raise MeaError(_lib.MEA_ERR_SHAPE, "q [B, Hq, D], k/v [T_k, Hkv, D]")
+    if not q.is_cuda:
+        raise MeaError(_lib.MEA_ERR_DEVICE, "tensors must live on the GPU")
+    _on_device(q.device, k=k, v=v)
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
     b, hq, d = q.shape
     tk, hkv, _ = k.shape
+    cu_seqlens_k = _check_cu("cu_seqlens_k", cu_seqlens_k, b + 1, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     ws_bytes = decode_workspace_size(b, tk, hq, hkv, d, split_keys)
@@ -209,14 +275,18 @@ def decode_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty_like(q)
+    else:
+        _check_buffer("out", out, (b, hq, d), q.dtype, q.device)
     if return_lse and lse is None:
         lse = torch.empty((hq, b), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check_buffer("lse", lse, (hq, b), torch.float32, q.device)
     if alibi_slopes is not None:
         alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
     rc = _lib.load().mea_decode_splitkv(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_k), b, tk,
         int(max_seqlen_k), hq, hkv, d, float(scale), _lib.MEA_MASK_CAUSAL, _ptr(alibi_slopes),
-        _dtype_code(q.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _dtype_code(q.dtype), _ptr(workspace), _check_workspace(workspace, q.device),
         int(split_keys), _stream(q.device))
     _lib.check(rc, "mea_decode_splitkv")
     return out, lse
@@ -239,8 +309,10 @@ def decode_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     n, hq, d = q.shape
     nb, bs, hkv, _ = k_cache.shape
     if v_cache.shape != k_cache.shape or block_table.dtype != torch.int32 \
-            or block_table.dim() != 2 or block_table.shape[0] != n:
+            or block_table.dim() != 2 or block_table.shape[0] != n or k_cache.shape[3] != d:
         raise MeaError(_lib.MEA_ERR_SHAPE, "cache / block table shapes disagree")
+    _on_device(q.device, k_cache=k_cache, v_cache=v_cache, block_table=block_table)
+    cu_seqlens_k = _check_cu("cu_seqlens_k", cu_seqlens_k, n + 1, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     total = int(total_k_bound) if total_k_bound is not None else nb * bs
@@ -249,15 +321,19 @@ def decode_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                                 dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty_like(q)
+    else:
+        _check_buffer("out", out, (n, hq, d), q.dtype, q.device)
     if lse is None:
         lse = torch.empty((hq, n), dtype=torch.float32, device=q.device)
+    else:
+        _check_buffer("lse", lse, (hq, n), torch.float32, q.device)
     if alibi_slopes is not None:
         alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
     rc = _lib.load().mea_decode_paged(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cu_seqlens_k), _ptr(out),
         _ptr(lse), n, nb, bs, block_table.shape[1], total, int(max_seqlen_k), hq, hkv, d,
         float(scale), _lib.MEA_MASK_CAUSAL, _ptr(alibi_slopes), _dtype_code(q.dtype),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), int(split_keys),
+        _ptr(workspace), _check_workspace(workspace, q.device), int(split_keys),
         _stream(q.device))
     _lib.check(rc, "mea_decode_paged")
     return out, lse
@@ -276,8 +352,20 @@ def decode_splitkv_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     the GPU share that array and race; keep them ordered on one stream. Raises ``MeaError`` with
     ``MEA_ERR_SCRATCH_LIMIT`` when the partials cannot fit in the array.
     """
+    if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape or k.shape[2] != q.shape[2]:
+        raise MeaError(_lib.MEA_ERR_SHAPE, "q [B, Hq, D], k/v [T_k, Hkv, D]")
+    if not q.is_cuda:
+        raise MeaError(_lib.MEA_ERR_DEVICE, "tensors must live on the GPU")
+    _on_device(q.device, k=k, v=v)
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
     b, hq, d = q.shape
     tk, hkv, _ = k.shape
+    cu_seqlens_k = _check_cu("cu_seqlens_k", cu_seqlens_k, b + 1, q.device)
+    _check_buffer("out", out, (b, hq, d), q.dtype, q.device)
+    if lse is not None:
+        _check_buffer("lse", lse, (hq, b), torch.float32, q.device)
+    if alibi_slopes is not None:
+        alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     rc = _lib.load().mea_decode_splitkv_noalloc(

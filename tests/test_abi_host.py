@@ -218,3 +218,57 @@ def test_python_binding_fails_loudly_without_gpu():
     cu = torch.tensor([0, 4], dtype=torch.int32)
     with pytest.raises(mea.MeaError):
         mea.attention_packed(q, q, q, cu, cu, 4)
+
+
+# ------------------------------------------------------------------ binding argument checks
+def test_binding_buffer_checks():
+    import torch
+    import memory_efficient_attention_b200 as mea
+    cpu = torch.device("cpu")
+    good = torch.zeros((4, 2, 64), dtype=torch.float16)
+    assert mea._check_buffer("out", good, (4, 2, 64), torch.float16, cpu) is good
+    for bad, shape, dtype in [(good, (4, 2, 32), torch.float16),       # wrong shape
+                              (good, (4, 2, 64), torch.bfloat16),      # wrong dtype
+                              (good.transpose(0, 1), (2, 4, 64), torch.float16)]:  # not contiguous
+        with pytest.raises(mea.MeaError) as e:
+            mea._check_buffer("out", bad, shape, dtype, cpu)
+        assert e.value.rc == _lib.MEA_ERR_SHAPE
+    with pytest.raises(mea.MeaError) as e:  # a host tensor where a device one is needed
+        mea._check_buffer("out", good, (4, 2, 64), torch.float16, torch.device("cuda", 0))
+    assert e.value.rc == _lib.MEA_ERR_SHAPE
+
+
+def test_binding_cu_seqlens_and_device_checks():
+    import torch
+    import memory_efficient_attention_b200 as mea
+    dev = torch.device("cuda", 0)
+    for bad in (torch.tensor([0, 4], dtype=torch.int64), torch.tensor([0, 4, 8], dtype=torch.int32)):
+        with pytest.raises(mea.MeaError) as e:
+            mea._check_cu("cu_seqlens_q", bad, 2, dev)
+        assert e.value.rc == _lib.MEA_ERR_SHAPE
+    with pytest.raises(mea.MeaError) as e:  # right shape, but host memory
+        mea._check_cu("cu_seqlens_q", torch.tensor([0, 4], dtype=torch.int32), 2, dev)
+    assert e.value.rc == _lib.MEA_ERR_DEVICE
+    with pytest.raises(mea.MeaError) as e:
+        mea._on_device(dev, k=torch.zeros(2))
+    assert e.value.rc == _lib.MEA_ERR_DEVICE
+    mea._on_device(dev, k=None)  # optional tensors are skipped
+    with pytest.raises(mea.MeaError) as e:
+        mea._check_workspace(torch.zeros(16, dtype=torch.uint8), dev)
+    assert e.value.rc == _lib.MEA_ERR_WORKSPACE
+
+
+def test_binding_decode_rejects_host_tensors_before_any_launch():
+    import torch
+    import memory_efficient_attention_b200 as mea
+    q = torch.zeros((2, 8, 64), dtype=torch.float16)
+    kv = torch.zeros((10, 2, 64), dtype=torch.float16)
+    cu = torch.tensor([0, 4, 10], dtype=torch.int32)
+    for call in (lambda: mea.decode_splitkv(q, kv, kv, cu, 6),
+                 lambda: mea.decode_splitkv_noalloc(q, kv, kv, cu, 6, out=torch.empty_like(q))):
+        with pytest.raises(mea.MeaError) as e:
+            call()
+        assert e.value.rc == _lib.MEA_ERR_DEVICE
+    with pytest.raises(mea.MeaError) as e:  # k and v shapes disagree
+        mea.decode_splitkv(q, kv, kv[:5], cu, 6)
+    assert e.value.rc == _lib.MEA_ERR_SHAPE
