@@ -76,3 +76,35 @@ def test_aggregate_is_units_of_all_ranks_over_slowest_time():
     import bench
     assert bench.aggregate_throughput(5.0, 1, 1000.0) == 5.0
     assert bench.aggregate_throughput(5.0, 4, 2000.0) == 10.0
+
+
+def test_reference_arm_line_has_the_contract_keys(monkeypatch, capsys):
+    """Rank 0 of `bench.py --impl reference` prints one JSON line with the bench keys, the
+    oracle's cpu_baseline and an e2e object with no host-device traffic (a tiny sample here)."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch
+    from mea_workloads import alibi_slope_values, make_qkv
+
+    def tiny(_target):
+        q, k, v = make_qkv([40, 24], [40, 24], 32, 8, 128, torch.bfloat16, 7)
+        return (q, k, v, [40, 24], alibi_slope_values(32).double(), 0.088), \
+            bench.fwd_flops([40, 24], 32, 128), "tiny sample"
+    monkeypatch.setattr(bench, "oracle_sample", tiny)
+    args = types.SimpleNamespace(impl="reference", gpus=1, steps=2, warmup=1,
+                                 decode_requests=64)
+    assert bench.run_reference(args, 1, 0) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["config"] == bench.step_config(args, 1)
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
