@@ -77,8 +77,9 @@ typedef enum {
  *   n_seqs        number of segments (>= 1); cu_seqlens_* hold n_seqs+1 entries each.
  *   total_q/k     T_q = cu_seqlens_q[n_seqs], T_k = cu_seqlens_k[n_seqs] (given by the caller
  *                 so that the host never reads device memory; they size the TMA views).
- *   max_seqlen_q  an upper bound on every L_q (sizes the work decomposition; rows past it are
- *                 not computed, so it must not be smaller than the true maximum).
+ *   max_seqlen_q  the largest L_q, or an upper bound on it. It only sizes the grid: every CTA
+ *                 reads the true lengths from cu_seqlens_q, so a smaller value still produces
+ *                 every row (more slowly, on fewer CTAs); 0 is treated as 1.
  *   scale         multiplies Q K^T before the bias (1/sqrt(D) is the usual choice).
  *   alibi_slopes  NULL, or DEVICE fp32 [n_heads_q] slopes (2^(-8(h+1)/Hq) is the usual choice).
  *   dtype         mea_dtype of q, k, v and out.
@@ -86,8 +87,9 @@ typedef enum {
  * MEA_ERR_HEADS also covers head counts so large that the kernel's integer head-block-to-group
  * mapping could round wrongly ((H/P - 1) * (R/P - 1) >= 2^32, with R = n_heads_q / n_heads_kv
  * and P its largest power-of-two divisor up to 128); no realistic head count reaches it.
- * Performance: cu_seqlens_q/k of up to 191 segments are kept in on-chip memory; longer lists
- * are read from global memory as the work is scheduled.
+ * Performance: the work items (a pair of query tiles of one segment and one block of query heads)
+ * are balanced over the GPU's SMs heaviest first; with up to 256 segments every CTA ranks them
+ * by length on chip, longer lists are walked in segment order (still complete, less balanced).
  */
 int mea_forward(const void* q, const void* k, const void* v, void* out, float* lse,
                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int n_seqs,
@@ -146,7 +148,10 @@ int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, f
  *     up to 256 bytes) cannot fit, the call returns MEA_ERR_SCRATCH_LIMIT and launches nothing.
  *   - The first call on a device looks up the array's device address on that device (one
  *     cudaGetSymbolAddress, with that device current); make that first call before any stream
- *     capture on that device.
+ *     capture on that device. The address belongs to the CUDA context that is current during
+ *     the call: it is remembered per device together with that context, and looked up again
+ *     (the same way) when a later call runs under another context of the device, for example
+ *     after cudaDeviceReset.
  *   - All calls share the one array and it keeps whatever the last call wrote. Nothing in it needs
  *     to start at zero (every partial is written before it is read). Two calls whose kernels
  *     overlap on the GPU (different streams, or different host threads, without ordering between

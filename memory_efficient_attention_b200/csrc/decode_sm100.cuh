@@ -36,6 +36,7 @@ struct DecParams {
   float* ws_lse;      // [n_slots, hq]
   int n_seqs;
   int hq;
+  int dh;             // head dim of q, k, v and out rows (<= D; the TMA zero-fills the rest)
   int R;              // query heads per KV head
   int RB;             // query heads per work item (<= 16, divides R)
   int n_hb;           // hq / RB
@@ -167,70 +168,62 @@ __global__ void __launch_bounds__(160, 1)
       const int nk = min(p.chunk, L - key0);
       const int n_tiles = (nk + C::BK - 1) / C::BK;
       const int g = (hb * p.RB) / p.R;
-      if (lane == 0) {
-        // Paged: the cache block ids of tile t+1 are loaded while tile t is being issued, so the
-        // table reads never wait in line behind the TMA issue.
-        constexpr int MAXPER = C::BK / 16;  // blocks per tile at the smallest block size
-        int ids_next[MAXPER] = {};
-        const int32_t* row = nullptr;
-        int per = 1, nblk = 0;
-        if constexpr (PAGED) {
-          row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-          per = p.block_size >= C::BK ? 1 : C::BK / p.block_size;
-          nblk = min((L + p.block_size - 1) / p.block_size, p.max_blocks);
-#pragma unroll
-          for (int i = 0; i < MAXPER; ++i) {
-            const int j = (key0 + i * p.block_size) / p.block_size;
-            ids_next[i] = (i < per && j < nblk) ? __ldg(row + j) : p.num_blocks;
-          }
-        }
+      if constexpr (PAGED) {
+        // Tile keys [kt, kt + 64) of request b come from `per` cache blocks: one box per block
+        // and per (K or V, 64-column atom) for block sizes 16 and 32 (boxes of block_size rows
+        // at row offsets that keep the 128-B swizzle aligned), or a 64-row slice of one block
+        // for block sizes that are multiples of 64. The boxes of a stage are issued by as many
+        // lanes, each of which also reads its block id one tile ahead (at 16-slot blocks a
+        // stage is 16 boxes of 2 KB, and one lane issuing them all starved the stream). Blocks
+        // past the request's last one use id num_blocks, which the TMA fills with zeros.
+        const int32_t* row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+        const int bs = p.block_size;
+        const int per = bs >= C::BK ? 1 : C::BK / bs;
+        const int nblk = min((L + bs - 1) / bs, p.max_blocks);
+        const int nbox = per * 2 * C::ATOMS;               // <= 16 boxes per stage
+        const int my_i = lane / (2 * C::ATOMS);            // block of the tile
+        const int my_v = (lane / C::ATOMS) & 1;            // K or V
+        const int my_a = lane % C::ATOMS;                  // 64-column atom
+        const bool issuer = lane < nbox;
+        auto block_id = [&](int t) {
+          const int j = (key0 + t * C::BK + my_i * bs) / bs;
+          return (issuer && t < n_tiles && j < nblk) ? __ldg(row + j) : p.num_blocks;
+        };
+        int id_next = block_id(0);
         for (int t = 0; t < n_tiles; ++t) {
-          int ids[MAXPER];
-#pragma unroll
-          for (int i = 0; i < MAXPER; ++i) ids[i] = ids_next[i];
-          if constexpr (PAGED) {
-            const int kn = key0 + (t + 1) * C::BK;
-#pragma unroll
-            for (int i = 0; i < MAXPER; ++i) {
-              const int j = (kn + i * p.block_size) / p.block_size;
-              ids_next[i] = (t + 1 < n_tiles && i < per && j < nblk) ? __ldg(row + j)
-                                                                       : p.num_blocks;
-            }
+          const int id = id_next;
+          id_next = block_id(t + 1);
+          const uint32_t s = cnt % C::NS;
+          const uint32_t ph = (cnt / C::NS) & 1u;
+          if (lane == 0) {
+            ok = mbar_wait(DBAR(B_E + s), ph ^ 1u, abort_flag, tmo, ecode | 1);
+            if (ok) mbar_arrive_expect_tx(DBAR(B_F + s), C::STAGE_BYTES);
           }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          if (issuer) {
+            const uint32_t dst = sbase + C::SMEM_RING + s * C::STAGE_BYTES +
+                                 my_v * C::KT_BYTES + my_a * C::ATOM_BYTES +
+                                 static_cast<uint32_t>(my_i * bs * 128);
+            const int r0 = bs >= C::BK ? (key0 + t * C::BK) % bs : 0;
+            tma_load_4d(dst, my_v ? &tm_v : &tm_k, DBAR(B_F + s), my_a * 64, g, r0, id);
+          }
+          ++cnt;
+        }
+      } else if (lane == 0) {
+        for (int t = 0; t < n_tiles; ++t) {
           const uint32_t s = cnt % C::NS;
           const uint32_t ph = (cnt / C::NS) & 1u;
           ok = mbar_wait(DBAR(B_E + s), ph ^ 1u, abort_flag, tmo, ecode | 1);
           if (!ok) break;
           mbar_arrive_expect_tx(DBAR(B_F + s), C::STAGE_BYTES);
           const uint32_t dst = sbase + C::SMEM_RING + s * C::STAGE_BYTES;
-          if constexpr (PAGED) {
-            // Tile keys [kt, kt + 64) of request b: one box per cache block (block sizes 16, 32:
-            // boxes of block_size rows at row offsets that keep the 128-B swizzle aligned) or a
-            // 64-row slice of one block (block sizes that are multiples of 64). Blocks past the
-            // request's last one use id num_blocks, which the TMA fills with zeros.
-            const int kt = key0 + t * C::BK;
-            const int bs = p.block_size;
-            const int r0 = bs >= C::BK ? kt % bs : 0;
+          const int tok = k0 + key0 + t * C::BK;
 #pragma unroll
-            for (int i = 0; i < MAXPER; ++i) {
-              if (i >= per) break;
-              const uint32_t rows_off = static_cast<uint32_t>(i * bs * 128);
-#pragma unroll
-              for (int a = 0; a < C::ATOMS; ++a) {
-                tma_load_4d(dst + a * C::ATOM_BYTES + rows_off, &tm_k, DBAR(B_F + s), a * 64, g,
-                            r0, ids[i]);
-                tma_load_4d(dst + C::KT_BYTES + a * C::ATOM_BYTES + rows_off, &tm_v,
-                            DBAR(B_F + s), a * 64, g, r0, ids[i]);
-              }
-            }
-          } else {
-            const int tok = k0 + key0 + t * C::BK;
-#pragma unroll
-            for (int a = 0; a < C::ATOMS; ++a) {
-              tma_load_3d(dst + a * C::ATOM_BYTES, &tm_k, DBAR(B_F + s), a * 64, g, tok);
-              tma_load_3d(dst + C::KT_BYTES + a * C::ATOM_BYTES, &tm_v, DBAR(B_F + s), a * 64,
-                          g, tok);
-            }
+          for (int a = 0; a < C::ATOMS; ++a) {
+            tma_load_3d(dst + a * C::ATOM_BYTES, &tm_k, DBAR(B_F + s), a * 64, g, tok);
+            tma_load_3d(dst + C::KT_BYTES + a * C::ATOM_BYTES, &tm_v, DBAR(B_F + s), a * 64,
+                        g, tok);
           }
           ++cnt;
         }
@@ -267,17 +260,20 @@ __global__ void __launch_bounds__(160, 1)
       // q fragments: rows g8 and g8+8 are heads hb*RB + row (zero when row >= RB).
       const int h_lo = hb * p.RB + g8, h_hi = hb * p.RB + g8 + 8;
       const bool v_lo = g8 < p.RB, v_hi = g8 + 8 < p.RB;
+      // Columns past dh are zero (as are the K/V columns the TMA fills past dh).
       uint32_t qa[D / 16][4];
       {
         const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
-        const size_t rlo = (static_cast<size_t>(b) * p.hq + h_lo) * (D / 2);
-        const size_t rhi = (static_cast<size_t>(b) * p.hq + h_hi) * (D / 2);
+        const int dw = p.dh >> 1;  // 32-bit words per row
+        const size_t rlo = (static_cast<size_t>(b) * p.hq + h_lo) * dw;
+        const size_t rhi = (static_cast<size_t>(b) * p.hq + h_hi) * dw;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          qa[kk][0] = v_lo ? __ldg(q32 + rlo + kk * 8 + t4) : 0u;
-          qa[kk][1] = v_hi ? __ldg(q32 + rhi + kk * 8 + t4) : 0u;
-          qa[kk][2] = v_lo ? __ldg(q32 + rlo + kk * 8 + 4 + t4) : 0u;
-          qa[kk][3] = v_hi ? __ldg(q32 + rhi + kk * 8 + 4 + t4) : 0u;
+          const bool c0 = kk * 8 + t4 < dw, c1 = kk * 8 + 4 + t4 < dw;
+          qa[kk][0] = (v_lo && c0) ? __ldg(q32 + rlo + kk * 8 + t4) : 0u;
+          qa[kk][1] = (v_hi && c0) ? __ldg(q32 + rhi + kk * 8 + t4) : 0u;
+          qa[kk][2] = (v_lo && c1) ? __ldg(q32 + rlo + kk * 8 + 4 + t4) : 0u;
+          qa[kk][3] = (v_hi && c1) ? __ldg(q32 + rhi + kk * 8 + 4 + t4) : 0u;
         }
       }
       float sl_lo = 0.f, sl_hi = 0.f;
@@ -488,7 +484,6 @@ __global__ void __launch_bounds__(256)
   const int c0 = s_start;
   using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   OutT* out = reinterpret_cast<OutT*>(p.out);
-  constexpr int D4 = D / 4;
   for (int rb = 0; rb < p.R; rb += 64) {  // heads of the group, 64 at a time
     const int rn = min(64, p.R - rb);
     for (int rr = warp; rr < rn; rr += 8) {
@@ -510,8 +505,9 @@ __global__ void __launch_bounds__(256)
       }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < rn * D4; idx += blockDim.x) {
-      const int rr = idx / D4, d = (idx - rr * D4) * 4;
+    const int dh4 = p.dh / 4;  // output columns (the partials hold D >= dh)
+    for (int idx = threadIdx.x; idx < rn * dh4; idx += blockDim.x) {
+      const int rr = idx / dh4, d = (idx - rr * dh4) * 4;
       const int head = g * p.R + rb + rr;
       const float m = s_m[rr], z = s_z[rr];
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -528,7 +524,7 @@ __global__ void __launch_bounds__(256)
         }
       }
       const float inv = z > 0.f ? 1.f / z : 0.f;
-      OutT* dst = out + (static_cast<size_t>(b) * p.hq + head) * D + d;
+      OutT* dst = out + (static_cast<size_t>(b) * p.hq + head) * p.dh + d;
       if constexpr (BF16) {
         reinterpret_cast<__nv_bfloat162*>(dst)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
         reinterpret_cast<__nv_bfloat162*>(dst)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);

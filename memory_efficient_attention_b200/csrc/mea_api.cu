@@ -65,8 +65,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 3-D tiled map over a row-major [d2, d1, d0] tensor of 16-bit elements, 128-byte swizzle.
 constexpr int kDtypeE4M3 = 2;  // internal: 8-bit e4m3 tensor (mea_forward_fp8)
 
-bool encode_3d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
-               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
+bool encode_3d_uncached(CUtensorMap* map, const void* base, int dtype, uint64_t d0,
+                        uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
   auto fn = encode_fn();
   if (!fn) return false;
   const uint64_t es = dtype == kDtypeE4M3 ? 1 : 2;
@@ -83,7 +83,69 @@ bool encode_3d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint6
   return r == CUDA_SUCCESS;
 }
 
+// ------------------------------------------------------------------------------------------
+// Cache of encoded tensor maps. A map only describes (address, sizes, strides, box, element
+// type, swizzle), so one encoded for the same arguments is the same 128 bytes; serving calls
+// that reuse their buffers (every decode step of a KV cache, for instance) skip the encoding.
+// The cache is the library's only state besides per-device attributes: kMapCache entries,
+// least recently used replaced first, guarded by a mutex.
+// ------------------------------------------------------------------------------------------
+struct MapKey {
+  const void* base;
+  int dtype, rank;
+  uint64_t dims[4];
+  uint32_t box[4];
+  bool operator==(const MapKey& o) const {
+    if (base != o.base || dtype != o.dtype || rank != o.rank) return false;
+    for (int i = 0; i < 4; ++i)
+      if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
+    return true;
+  }
+};
+constexpr int kMapCache = 64;
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  uint64_t used[kMapCache] = {};  // 0 = empty slot
+  uint64_t tick = 0;
+  std::mutex mu;
+};
+MapCache g_maps;
+
+// Copies the cached map for `k` into *out; false when it is not cached.
+bool map_lookup(const MapKey& k, CUtensorMap* out) {
+  std::lock_guard<std::mutex> lk(g_maps.mu);
+  for (int i = 0; i < kMapCache; ++i)
+    if (g_maps.used[i] && g_maps.key[i] == k) {
+      g_maps.used[i] = ++g_maps.tick;
+      *out = g_maps.map[i];
+      return true;
+    }
+  return false;
+}
+
+void map_insert(const MapKey& k, const CUtensorMap& m) {
+  std::lock_guard<std::mutex> lk(g_maps.mu);
+  int victim = 0;
+  for (int i = 0; i < kMapCache; ++i) {
+    if (g_maps.used[i] == 0) {
+      victim = i;
+      break;
+    }
+    if (g_maps.used[i] < g_maps.used[victim]) victim = i;
+  }
+  g_maps.key[victim] = k;
+  g_maps.map[victim] = m;
+  g_maps.used[victim] = ++g_maps.tick;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Head dims of the forward: a multiple of 8 from 8 to 128 for 16-bit inputs (16-byte rows), a
+// multiple of 16 from 16 to 128 for e4m3 inputs.
+bool fwd_head_dim_ok(int d, bool e8) {
+  return e8 ? (d >= 16 && d <= 128 && d % 16 == 0) : (d >= 8 && d <= 128 && d % 8 == 0);
+}
 
 int largest_pow2_divisor(int x, int cap) {
   int p = 1;
@@ -91,63 +153,70 @@ int largest_pow2_divisor(int x, int cap) {
   return p;
 }
 
-// Constants of the forward kernel's division-free schedule (see FwdParams): shifts for the
-// power-of-two packing factors, the multiplier that maps a head block to its KV group, and the
-// per-CTA stride through the item list in mixed radix (t_max, n_seqs, n_hb).
-// Returns false when (hb * g_mul) >> 32 would not be exact for every head block
-// ((n_hb - 1) * (d - 1) < 2^32 is sufficient).
-static bool fwd_schedule_constants(mea::FwdParams& p, int grid) {
+// Shifts for the power-of-two packing factors and the multiplier that maps a head block to its
+// KV group (see FwdParams). Returns false when (hb * g_mul) >> 32 would not be exact for every
+// head block ((n_hb - 1) * (d - 1) < 2^32 is sufficient).
+static bool fwd_schedule_constants(mea::FwdParams& p) {
   int l2p = 0;
   while ((1 << l2p) < p.P) ++l2p;
   int l2t = 0;
-  while ((1 << l2t) < 2 * p.tok_per_tile) ++l2t;
+  while ((1 << l2t) < p.subtiles * p.tok_per_tile) ++l2t;
   p.log2_p = l2p;
   p.log2_tpp = l2t;
   const unsigned long long d = static_cast<unsigned long long>(p.R / p.P);
   p.g_mul = ((1ull << 32) + d - 1) / d;
-  if (static_cast<unsigned long long>(p.n_hb - 1) * (d - 1) >= (1ull << 32)) return false;
-  const long long per = static_cast<long long>(p.n_seqs) * p.n_hb;
-  const long long g = grid;
-  p.step_tr = static_cast<int>(g / per);
-  const long long r = g % per;
-  p.step_seg = static_cast<int>(r / p.n_hb);
-  p.step_hb = static_cast<int>(r % p.n_hb);
-  return true;
+  return static_cast<unsigned long long>(p.n_hb - 1) * (d - 1) < (1ull << 32);
 }
+
+// cudaFuncSetAttribute(max dynamic shared memory) once per (kernel, device); the result of that
+// one call is kept and returned on every later call, so a failure is never forgotten. The kernel
+// is a template argument so that every kernel (not every kernel signature) has its own state.
+template <auto kern>
+cudaError_t smem_attr_once(uint32_t smem) {
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t result[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    result[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  return result[dev];
+}
+
+// Drops a launch error left by an earlier, unrelated call, so that the check after this
+// call's launches reports only their own failures.
+inline void clear_stale_launch_error() { (void)cudaGetLastError(); }
 
 // ------------------------------------------------------------------------------------------
 // Forward launch dispatch.
 // ------------------------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool ALIBI, bool E8 = false>
 int launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                 const mea::FwdParams& p, int grid, cudaStream_t stream) {
-  auto kern = mea::mea_fwd_sm100_kernel<D, BF16, CAUSAL, ALIBI, E8>;
+                 const CUtensorMap& to, const mea::FwdParams& p, int grid, cudaStream_t stream) {
+  constexpr auto kern = mea::mea_fwd_sm100_kernel<D, BF16, CAUSAL, ALIBI, E8>;
   constexpr uint32_t smem = mea::FwdCfg<D, E8>::SMEM_TOTAL;
-  static std::once_flag once[kMaxDevices];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  cudaError_t attr_err = cudaSuccess;
-  std::call_once(once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr_err != cudaSuccess) return MEA_ERR_CUDA;
-  kern<<<grid, mea::FwdCfg<D>::THREADS, smem, stream>>>(tq, tk, tv, p);
+  if (smem_attr_once<kern>(smem) != cudaSuccess) return MEA_ERR_CUDA;
+  clear_stale_launch_error();
+  kern<<<grid, mea::FwdCfg<D>::THREADS, smem, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
 
 template <int D, bool BF16, bool E8 = false>
 int launch_fwd_d(bool causal, bool alibi, const CUtensorMap& tq, const CUtensorMap& tk,
-                 const CUtensorMap& tv, const mea::FwdParams& p, int grid, cudaStream_t s) {
+                 const CUtensorMap& tv, const CUtensorMap& to, const mea::FwdParams& p, int grid,
+                 cudaStream_t s) {
   if (causal)
-    return alibi ? launch_fwd_t<D, BF16, true, true, E8>(tq, tk, tv, p, grid, s)
-                 : launch_fwd_t<D, BF16, true, false, E8>(tq, tk, tv, p, grid, s);
-  return alibi ? launch_fwd_t<D, BF16, false, true, E8>(tq, tk, tv, p, grid, s)
-               : launch_fwd_t<D, BF16, false, false, E8>(tq, tk, tv, p, grid, s);
+    return alibi ? launch_fwd_t<D, BF16, true, true, E8>(tq, tk, tv, to, p, grid, s)
+                 : launch_fwd_t<D, BF16, true, false, E8>(tq, tk, tv, to, p, grid, s);
+  return alibi ? launch_fwd_t<D, BF16, false, true, E8>(tq, tk, tv, to, p, grid, s)
+               : launch_fwd_t<D, BF16, false, false, E8>(tq, tk, tv, to, p, grid, s);
 }
 
 // 4-D tiled map over a paged cache [d3 blocks, d2 slots, d1 heads, d0] of 16-bit elements.
-bool encode_4d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
-               uint64_t d2, uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+bool encode_4d_uncached(CUtensorMap* map, const void* base, int dtype, uint64_t d0,
+                        uint64_t d1, uint64_t d2, uint64_t d3, uint32_t b0, uint32_t b1,
+                        uint32_t b2, uint32_t b3) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {d0, d1, d2, d3};
@@ -162,20 +231,28 @@ bool encode_4d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint6
   return r == CUDA_SUCCESS;
 }
 
+// 3-D / 4-D maps through the cache (same arguments as the uncached encoders).
+bool encode_3d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  const MapKey k{base, dtype, 3, {d0, d1, d2, 0}, {b0, b1, b2, 0}};
+  if (map_lookup(k, map)) return true;
+  if (!encode_3d_uncached(map, base, dtype, d0, d1, d2, b0, b1, b2)) return false;
+  map_insert(k, *map);
+  return true;
+}
+
+bool encode_4d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  const MapKey k{base, dtype, 4, {d0, d1, d2, d3}, {b0, b1, b2, b3}};
+  if (map_lookup(k, map)) return true;
+  if (!encode_4d_uncached(map, base, dtype, d0, d1, d2, d3, b0, b1, b2, b3)) return false;
+  map_insert(k, *map);
+  return true;
+}
+
 // ------------------------------------------------------------------------------------------
 // Backward launch dispatch.
 // ------------------------------------------------------------------------------------------
-template <typename K>
-bool set_smem_once(K kern, uint32_t smem, std::once_flag (&once)[kMaxDevices]) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  cudaError_t err = cudaSuccess;
-  std::call_once(once[dev], [&] {
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  return err == cudaSuccess;
-}
-
 struct BwdMaps {
   CUtensorMap q, dout, k, v;  // 128-row boxes of one head
 };
@@ -184,11 +261,11 @@ template <int D, bool BF16, bool CAUSAL, bool ALIBI>
 int launch_bwd_t(const BwdMaps& m, const mea::BwdParams& p, int max_q, int max_k,
                  cudaStream_t stream) {
   constexpr uint32_t smem = mea::BwdTcCfg<D>::SMEM_TOTAL;
-  auto kdkdv = mea::mea_bwd_dkdv_tc_kernel<D, BF16, CAUSAL, ALIBI>;
-  auto kdq = mea::mea_bwd_dq_tc_kernel<D, BF16, CAUSAL, ALIBI>;
-  static std::once_flag once_a[kMaxDevices], once_b[kMaxDevices];
-  if (!set_smem_once(kdkdv, smem, once_a) || !set_smem_once(kdq, smem, once_b))
+  constexpr auto kdkdv = mea::mea_bwd_dkdv_tc_kernel<D, BF16, CAUSAL, ALIBI>;
+  constexpr auto kdq = mea::mea_bwd_dq_tc_kernel<D, BF16, CAUSAL, ALIBI>;
+  if (smem_attr_once<kdkdv>(smem) != cudaSuccess || smem_attr_once<kdq>(smem) != cudaSuccess)
     return MEA_ERR_CUDA;
+  clear_stale_launch_error();
   const unsigned long long tmo = g_timeout_ns.load();
   const long long rows = static_cast<long long>(p.total_q) * p.hq;
   if (rows > 0)
@@ -218,16 +295,10 @@ int launch_bwd_d(bool causal, bool alibi, const BwdMaps& m, const mea::BwdParams
 template <int D, bool BF16, bool ALIBI, bool PAGED>
 int launch_dec_t(const CUtensorMap& tk, const CUtensorMap& tv, const mea::DecParams& p,
                  int grid, int n_kv_heads, cudaStream_t stream) {
-  auto kern = mea::mea_decode_split_kernel<D, BF16, ALIBI, PAGED>;
+  constexpr auto kern = mea::mea_decode_split_kernel<D, BF16, ALIBI, PAGED>;
   constexpr uint32_t smem = mea::DecCfg<D>::SMEM_TOTAL;
-  static std::once_flag once[kMaxDevices];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  cudaError_t attr_err = cudaSuccess;
-  std::call_once(once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr_err != cudaSuccess) return MEA_ERR_CUDA;
+  if (smem_attr_once<kern>(smem) != cudaSuccess) return MEA_ERR_CUDA;
+  clear_stale_launch_error();
   if (grid > 0) kern<<<grid, mea::DecCfg<D>::THREADS, smem, stream>>>(tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return MEA_ERR_CUDA;
   dim3 mgrid(p.n_seqs, n_kv_heads);
@@ -264,10 +335,15 @@ struct DecLayout {
   size_t o_bytes = 0, lse_off = 0, total = 0;
 };
 
+// Head dims of the decode: a multiple of 8 from 8 to 128; the kernels run 64 or 128 wide.
+bool dec_head_dim_ok(int d) { return d >= 8 && d <= 128 && d % 8 == 0; }
+int padded_head_dim(int d) { return d <= 64 ? 64 : 128; }
+
 bool dec_layout(int n_seqs, int total_k, int hq, int hkv, int d, int split_keys, int sms,
                 DecLayout& L) {
-  if (n_seqs < 1 || total_k < 0 || hq < 1 || hkv < 1 || hq % hkv || (d != 64 && d != 128))
+  if (n_seqs < 1 || total_k < 0 || hq < 1 || hkv < 1 || hq % hkv || !dec_head_dim_ok(d))
     return false;
+  d = padded_head_dim(d);  // the partials are kept at the kernel's width
   if (split_keys < 0 || split_keys % 64) return false;
   const int R = hq / hkv;
   const int n_hb = hq / decode_rb(R);
@@ -294,21 +370,49 @@ static __device__ __align__(256) unsigned char mea_noalloc_scratch[MEA_DECODE_NO
 
 namespace {
 
-void* g_noalloc_addr[kMaxDevices] = {};
-cudaError_t g_noalloc_err[kMaxDevices] = {};
-std::once_flag g_noalloc_once[kMaxDevices];
+PFN_cuCtxGetCurrent_v4000 ctx_current_fn() {
+  static PFN_cuCtxGetCurrent_v4000 fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuCtxGetCurrent_v4000>(nullptr);
+    return reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+  }();
+  return fn;
+}
 
-// Device address of mea_noalloc_scratch on the current device (looked up on first use).
+// The device address of mea_noalloc_scratch belongs to the CUDA context that was current when
+// it was looked up (a device can carry several contexts, and a context can be destroyed and
+// recreated). It is cached per device together with that context and looked up again
+// whenever a call runs under another one.
+struct NoallocAddr {
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
+NoallocAddr g_noalloc[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of mea_noalloc_scratch for the current device and context.
 int noalloc_scratch_address(void** ptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MEA_ERR_CUDA;
-  std::call_once(g_noalloc_once[dev], [dev] {
+  auto get_ctx = ctx_current_fn();
+  if (!get_ctx) return MEA_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return MEA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  NoallocAddr& e = g_noalloc[dev];
+  if (ctx == nullptr || e.ctx != ctx || e.addr == nullptr) {
+    // The lookup makes the device's primary context current when no context is yet.
     void* p = nullptr;
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, mea_noalloc_scratch);
-    g_noalloc_addr[dev] = p;
-  });
-  if (g_noalloc_err[dev] != cudaSuccess || g_noalloc_addr[dev] == nullptr) return MEA_ERR_CUDA;
-  *ptr = g_noalloc_addr[dev];
+    if (cudaGetSymbolAddress(&p, mea_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return MEA_ERR_CUDA;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return MEA_ERR_CUDA;
+    e.ctx = ctx;
+    e.addr = p;
+  }
+  *ptr = e.addr;
   return MEA_OK;
 }
 
@@ -345,8 +449,8 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, float* 
   if (n_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_q > total_q)
     return MEA_ERR_SHAPE;
   if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
-  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
-  if (e8 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  // Rows of 16-bit elements need a multiple of 16 bytes (TMA strides); e4m3 rows the same.
+  if (!fwd_head_dim_ok(head_dim, e8)) return MEA_ERR_HEAD_DIM;
   if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
   if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
   if (!std::isfinite(scale) || !std::isfinite(qk_descale) || !std::isfinite(v_descale))
@@ -357,7 +461,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, float* 
     return MEA_ERR_ALIGN;
   DeviceInfo di;
   if (int rc = current_device_info(di); rc != MEA_OK) return rc;
-  if (total_q == 0 || max_seqlen_q == 0) return MEA_OK;
+  if (total_q == 0) return MEA_OK;
 
   const int R = n_heads_q / n_heads_kv;
   const int P = largest_pow2_divisor(R, 128);
@@ -370,37 +474,50 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, float* 
   p.n_seqs = n_seqs;
   p.total_q = total_q;
   p.hq = n_heads_q;
+  p.dh = head_dim;
   p.P = P;
   p.R = R;
   p.n_hb = n_heads_q / P;
   p.tok_per_tile = 128 / P;
-  p.t_max = (max_seqlen_q + 2 * p.tok_per_tile - 1) / (2 * p.tok_per_tile);
-  p.n_items = static_cast<long long>(p.t_max) * n_seqs * p.n_hb;
+  p.subtiles = 2;
   p.c1 = scale * qk_descale * 1.4426950408889634f;
   p.o_scale = v_descale;
   p.timeout_ns = g_timeout_ns.load();
+  if (!fwd_schedule_constants(p)) return MEA_ERR_HEADS;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const uint64_t tk_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
   const int in_dtype = e8 ? kDtypeE4M3 : dtype;
   const uint32_t box0 = e8 ? 128 : 64;  // elements per 128-byte swizzle row
+  // out: one warp's 32 rows (32/P tokens x P heads, or 32 of the P heads of one token).
+  const uint32_t out_heads = P < 32 ? static_cast<uint32_t>(P) : 32u;
+  const uint32_t out_toks = P < 32 ? static_cast<uint32_t>(32 / P) : 1u;
   if (!encode_3d(&tq, q, in_dtype, head_dim, n_heads_q, total_q, box0, P, 128 / P) ||
       !encode_3d(&tk, k, in_dtype, head_dim, n_heads_kv, tk_rows, box0, 1, 128) ||
-      !encode_3d(&tv, v, in_dtype, head_dim, n_heads_kv, tk_rows, box0, 1, 128))
+      !encode_3d(&tv, v, in_dtype, head_dim, n_heads_kv, tk_rows, box0, 1, 128) ||
+      !encode_3d(&to, out, dtype, head_dim, n_heads_q, total_q, 64, out_heads, out_toks))
     return MEA_ERR_CUDA;
-  const int grid = static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms);
-  if (!fwd_schedule_constants(p, grid)) return MEA_ERR_HEADS;
+  // Every CTA walks the live items of the whole problem; max_seqlen_q only bounds how many
+  // can exist, so a grid wider than that would leave CTAs idle.
+  const long long pairs_max = (static_cast<long long>(max_seqlen_q) + 2 * p.tok_per_tile - 1) /
+                              (2 * p.tok_per_tile);
+  const long long items_max = pairs_max * n_seqs * p.n_hb;
+  const int grid = static_cast<int>(items_max < di.sms ? (items_max > 0 ? items_max : 1) : di.sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool causal = mask_kind == MEA_MASK_CAUSAL;
   const bool alibi = alibi_slopes != nullptr;
   if (e8)
-    return dtype == MEA_BF16 ? launch_fwd_d<128, true, true>(causal, alibi, tq, tk, tv, p, grid, s)
-                             : launch_fwd_d<128, false, true>(causal, alibi, tq, tk, tv, p, grid, s);
-  if (head_dim == 128)
-    return dtype == MEA_BF16 ? launch_fwd_d<128, true>(causal, alibi, tq, tk, tv, p, grid, s)
-                             : launch_fwd_d<128, false>(causal, alibi, tq, tk, tv, p, grid, s);
-  return dtype == MEA_BF16 ? launch_fwd_d<64, true>(causal, alibi, tq, tk, tv, p, grid, s)
-                           : launch_fwd_d<64, false>(causal, alibi, tq, tk, tv, p, grid, s);
+    return dtype == MEA_BF16
+               ? launch_fwd_d<128, true, true>(causal, alibi, tq, tk, tv, to, p, grid, s)
+               : launch_fwd_d<128, false, true>(causal, alibi, tq, tk, tv, to, p, grid, s);
+  // Head dims below 64 run in the 64-wide kernel, those up to 128 in the 128-wide one: the TMA
+  // loads fill the columns past head_dim with zeros (they add nothing to Q K^T and give zero
+  // columns of O, which no store writes).
+  if (head_dim > 64)
+    return dtype == MEA_BF16 ? launch_fwd_d<128, true>(causal, alibi, tq, tk, tv, to, p, grid, s)
+                             : launch_fwd_d<128, false>(causal, alibi, tq, tk, tv, to, p, grid, s);
+  return dtype == MEA_BF16 ? launch_fwd_d<64, true>(causal, alibi, tq, tk, tv, to, p, grid, s)
+                           : launch_fwd_d<64, false>(causal, alibi, tq, tk, tv, to, p, grid, s);
 }
 
 extern "C" {
@@ -413,7 +530,8 @@ const char* mea_status_string(int status) {
     case MEA_ERR_NULL: return "MEA_ERR_NULL: a required pointer is NULL";
     case MEA_ERR_SHAPE: return "MEA_ERR_SHAPE: invalid sizes";
     case MEA_ERR_HEADS: return "MEA_ERR_HEADS: n_heads_q must be a positive multiple of n_heads_kv";
-    case MEA_ERR_HEAD_DIM: return "MEA_ERR_HEAD_DIM: head_dim must be 64 or 128";
+    case MEA_ERR_HEAD_DIM:
+      return "MEA_ERR_HEAD_DIM: head_dim is not supported by this entry point (see mea.h)";
     case MEA_ERR_DTYPE: return "MEA_ERR_DTYPE: dtype must be MEA_F16 or MEA_BF16";
     case MEA_ERR_ALIGN: return "MEA_ERR_ALIGN: tensor base pointers must be 16-byte aligned";
     case MEA_ERR_MASK: return "MEA_ERR_MASK: mask_kind is not a mea_mask value";
@@ -448,6 +566,7 @@ int mea_device_error(int* code, int clear) {
 
 int mea_wait_selftest(unsigned long long timeout_ns, int arrive, void* stream) {
   const unsigned long long t = timeout_ns ? timeout_ns : g_timeout_ns.load();
+  clear_stale_launch_error();
   mea::mea_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(t, arrive);
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
@@ -568,7 +687,7 @@ int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, f
     return MEA_ERR_SHAPE;
   if (split_keys < 0 || split_keys % 64) return MEA_ERR_SHAPE;
   if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
-  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (!dec_head_dim_ok(head_dim)) return MEA_ERR_HEAD_DIM;
   if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
   if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
   if (!std::isfinite(scale)) return MEA_ERR_SCALE;
@@ -600,6 +719,7 @@ int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, f
   p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.lse_off);
   p.n_seqs = n_seqs;
   p.hq = n_heads_q;
+  p.dh = head_dim;
   p.R = R;
   p.RB = decode_rb(R);
   p.n_hb = n_heads_q / p.RB;
@@ -617,7 +737,7 @@ int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, f
   const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool alibi = alibi_slopes != nullptr;
-  if (head_dim == 128)
+  if (head_dim > 64)
     return dtype == MEA_BF16 ? launch_dec_d<128, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
                              : launch_dec_d<128, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
   return dtype == MEA_BF16 ? launch_dec_d<64, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
@@ -638,7 +758,7 @@ int mea_decode_paged(const void* q, const void* k_cache, const void* v_cache,
     return MEA_ERR_SHAPE;
   if (split_keys < 0 || split_keys % 64) return MEA_ERR_SHAPE;
   if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
-  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (!dec_head_dim_ok(head_dim)) return MEA_ERR_HEAD_DIM;
   if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
   if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
   if (!std::isfinite(scale)) return MEA_ERR_SCALE;
@@ -672,6 +792,7 @@ int mea_decode_paged(const void* q, const void* k_cache, const void* v_cache,
   p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.lse_off);
   p.n_seqs = n_seqs;
   p.hq = n_heads_q;
+  p.dh = head_dim;
   p.R = R;
   p.RB = decode_rb(R);
   p.n_hb = n_heads_q / p.RB;
@@ -691,7 +812,7 @@ int mea_decode_paged(const void* q, const void* k_cache, const void* v_cache,
   const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool alibi = alibi_slopes != nullptr;
-  if (head_dim == 128)
+  if (head_dim > 64)
     return dtype == MEA_BF16
                ? launch_dec_d<128, true, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
                : launch_dec_d<128, false, true>(alibi, tk, tv, p, grid, n_heads_kv, s);
@@ -709,7 +830,7 @@ int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void
     return MEA_ERR_SHAPE;
   if (split_keys < 0 || split_keys % 64) return MEA_ERR_SHAPE;
   if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
-  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (!dec_head_dim_ok(head_dim)) return MEA_ERR_HEAD_DIM;
   if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
   if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
   if (!std::isfinite(scale)) return MEA_ERR_SCALE;
@@ -753,6 +874,7 @@ int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void
   p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(scratch) + L.lse_off);
   p.n_seqs = n_seqs;
   p.hq = n_heads_q;
+  p.dh = head_dim;
   p.R = R;
   p.RB = decode_rb(R);
   p.n_hb = n_heads_q / p.RB;
@@ -770,7 +892,7 @@ int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void
   const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool alibi = alibi_slopes != nullptr;
-  if (head_dim == 128)
+  if (head_dim > 64)
     return dtype == MEA_BF16 ? launch_dec_d<128, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
                              : launch_dec_d<128, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
   return dtype == MEA_BF16 ? launch_dec_d<64, true>(alibi, tk, tv, p, grid, n_heads_kv, s)

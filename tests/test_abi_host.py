@@ -67,8 +67,9 @@ def fwd(lib, **kw):
     (dict(max_q=9), _lib.MEA_ERR_SHAPE),
     (dict(hq=6, hkv=4), _lib.MEA_ERR_HEADS),
     (dict(hkv=0), _lib.MEA_ERR_HEADS),
-    (dict(d=96), _lib.MEA_ERR_HEAD_DIM),
-    (dict(d=256), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=100), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=136), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=0), _lib.MEA_ERR_HEAD_DIM),
     (dict(dtype=2), _lib.MEA_ERR_DTYPE),
     (dict(mask=2), _lib.MEA_ERR_MASK),
     (dict(scale=float("nan")), _lib.MEA_ERR_SCALE),
@@ -99,7 +100,8 @@ def dec(lib, **kw):
     (dict(max_k=101), _lib.MEA_ERR_SHAPE),
     (dict(split=100), _lib.MEA_ERR_SHAPE),
     (dict(hq=12, hkv=8), _lib.MEA_ERR_HEADS),
-    (dict(d=32), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=36), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=256), _lib.MEA_ERR_HEAD_DIM),
     (dict(dtype=-1), _lib.MEA_ERR_DTYPE),
     (dict(mask=3), _lib.MEA_ERR_MASK),
     (dict(v=A + 4), _lib.MEA_ERR_ALIGN),
@@ -193,7 +195,8 @@ def paged(lib, **kw):
     (dict(max_k=161), _lib.MEA_ERR_SHAPE),
     (dict(split=100), _lib.MEA_ERR_SHAPE),
     (dict(hq=12, hkv=8), _lib.MEA_ERR_HEADS),
-    (dict(d=80), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=84), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=192), _lib.MEA_ERR_HEAD_DIM),
     (dict(dtype=7), _lib.MEA_ERR_DTYPE),
     (dict(table=A + 2), _lib.MEA_ERR_ALIGN),
     (dict(vc=A + 8), _lib.MEA_ERR_ALIGN),

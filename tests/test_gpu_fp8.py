@@ -31,11 +31,11 @@ def _quantized(shape, seed, descale):
     return x.to(torch.float8_e4m3fn)
 
 
-def _case(seqlens, hq, hkv, causal, alibi, scale, seed, out_dtype=torch.bfloat16):
+def _case(seqlens, hq, hkv, causal, alibi, scale, seed, out_dtype=torch.bfloat16, d=128):
     tq = sum(seqlens)
-    q8 = _quantized((tq, hq, 128), seed, QD)
-    k8 = _quantized((tq, hkv, 128), seed + 1, KD)
-    v8 = _quantized((tq, hkv, 128), seed + 2, VD)
+    q8 = _quantized((tq, hq, d), seed, QD)
+    k8 = _quantized((tq, hkv, d), seed + 1, KD)
+    v8 = _quantized((tq, hkv, d), seed + 2, VD)
     slopes = alibi_slope_values(hq) if alibi else None
     cu = cu_seqlens(seqlens)
     out, lse = mea.attention_packed_fp8(q8.cuda(), k8.cuda(), v8.cuda(), cu.cuda(), cu.cuda(),
@@ -95,8 +95,13 @@ def test_fp8_half_output_and_longer_segments():
     _case([1000, 700], 8, 2, True, True, 1 / math.sqrt(128), 1530, out_dtype=torch.float16)
 
 
+@pytest.mark.parametrize("d", [16, 64, 96])
+def test_fp8_other_head_dims(d):
+    _case([130, 77, 300], 8, 2, True, True, 1 / math.sqrt(d), 1540 + d, d=d)
+
+
 def test_fp8_rejects_other_head_dims_and_dtypes():
-    x = torch.zeros((4, 2, 64), dtype=torch.float8_e4m3fn, device="cuda")
+    x = torch.zeros((4, 2, 72), dtype=torch.float8_e4m3fn, device="cuda")
     cu = torch.tensor([0, 4], dtype=torch.int32, device="cuda")
     with pytest.raises(mea.MeaError):
         mea.attention_packed_fp8(x, x, x, cu, cu, 4)

@@ -146,7 +146,10 @@ def test_workload4_decode_sampled():
     # oracle on a seeded sample of requests (all their heads), copied back to the host
     import numpy as np
     rng = np.random.default_rng(w.seed)
-    reqs = sorted(set(int(x) for x in rng.choice(len(w.seqlens_k), 8, replace=False)))
+    reqs = set(int(x) for x in rng.choice(len(w.seqlens_k), 8, replace=False))
+    # always the longest request (the most chunks) and the shortest one
+    reqs |= {int(np.argmax(w.seqlens_k)), int(np.argmin(w.seqlens_k))}
+    reqs = sorted(reqs)
     for b in reqs:
         a, e = int(cu_k[b]), int(cu_k[b + 1])
         ro, rl = oracle.decode(q[b:b + 1].cpu(), k[a:e].cpu(), v[a:e].cpu(), [0, e - a], w.scale)
@@ -163,19 +166,27 @@ def test_tile_edges(lens, causal):
 
 
 @pytest.mark.parametrize("hq,hkv", [(1, 1), (2, 1), (4, 1), (8, 1), (16, 2), (8, 8), (32, 2),
-                                    (6, 2), (12, 4), (3, 1), (128, 1), (256, 2)])
+                                    (6, 2), (12, 4), (3, 1), (64, 1), (128, 1), (256, 2)])
 def test_gqa_packing(hq, hkv):
     lens = [70, 200, 33]
     check_packed(lens, lens, hq, hkv, 64, torch.bfloat16, True, hq <= 32, 0.125, 100 + hq)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [32, 64, 96, 128])
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("causal,alibi", [(False, False), (True, False), (True, True),
                                           (False, True)])
 def test_dtypes_dims_masks(d, dtype, causal, alibi):
     lens = [190, 1, 64, 385]
     check_packed(lens, lens, 8, 2, d, dtype, causal, alibi, 1.0 / math.sqrt(d), 300 + d)
+
+
+@pytest.mark.parametrize("d", [8, 16, 40, 72, 80, 120])
+def test_other_head_dims(d):
+    # any multiple of 8 up to 128: the 64- or 128-wide kernel with zero-filled columns
+    lens = [130, 7, 300]
+    check_packed(lens, lens, 8, 2, d, torch.bfloat16, True, True, 1.0 / math.sqrt(d), 350 + d)
+    check_packed(lens, lens, 4, 4, d, torch.float16, False, False, 1.0 / math.sqrt(d), 351 + d)
 
 
 def test_lq_ne_lk_bottom_right_and_empty():
@@ -186,18 +197,49 @@ def test_lq_ne_lk_bottom_right_and_empty():
         check_packed(lq, lk, 8, 4, 128, torch.bfloat16, causal, True, 0.09, 77)
 
 
-@pytest.mark.parametrize("n_seqs", [191, 192, 300])
-def test_many_segments(n_seqs):
-    # the forward keeps cu_seqlens in shared memory for up to 191 segments and reads them from
-    # global memory beyond that; both sides of the limit, causal with GQA (R = 3)
+@pytest.mark.parametrize("n_seqs", [255, 256, 257, 300, 1000])
+@pytest.mark.parametrize("causal", [False, True])
+def test_many_segments(n_seqs, causal):
+    # the forward ranks up to 256 segments by length on chip and walks longer lists in segment
+    # order; both sides of the limit, with GQA (R = 3) and some empty segments
     g = torch.Generator().manual_seed(n_seqs)
-    lens = torch.randint(1, 161, (n_seqs,), generator=g).tolist()
-    check_packed(lens, lens, 6, 2, 64, torch.float16, True, False, 0.125, 900 + n_seqs)
+    lens = torch.randint(0, 161, (n_seqs,), generator=g).tolist()
+    lens[0] = max(lens[0], 1)
+    check_packed(lens, lens, 6, 2, 64, torch.float16, causal, False, 0.125, 900 + n_seqs)
 
 
 def test_max_seqlen_upper_bound():
     lens = [50, 20]
     check_packed(lens, lens, 4, 2, 64, torch.float16, True, False, 0.125, 5, max_seqlen_q=70)
+
+
+@pytest.mark.parametrize("max_seqlen_q", [1, 100])
+def test_max_seqlen_below_true_maximum_still_complete(max_seqlen_q):
+    # max_seqlen_q only sizes the grid: every row is produced from the true lengths
+    lens = [700, 3, 260]
+    check_packed(lens, lens, 8, 2, 128, torch.bfloat16, True, True, 0.09, 6,
+                 max_seqlen_q=max_seqlen_q)
+
+
+def test_out_16_byte_offset():
+    # out 16-byte but not 32-byte aligned: whole tiles still go through TMA stores (which need
+    # 16 bytes), partial ones through the 16-byte store path
+    lens = [100, 37]
+    hq, hkv, d, dtype = 8, 2, 128, torch.bfloat16
+    q, k, v = make_qkv(lens, lens, hq, hkv, d, dtype, 31)
+    cu = cu_seqlens(lens)
+    n = q.numel()
+    buf = torch.full((n + 8 + CANARY,), float("nan"), dtype=dtype, device="cuda")
+    buf[n + 8:] = 7.0
+    out = buf[8:n + 8].view(q.shape)
+    assert out.data_ptr() % 32 == 16
+    mea.attention_packed(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), cu.cuda(), 100, causal=True,
+                         scale=0.09, out=out)
+    torch.cuda.synchronize()
+    assert torch.isnan(buf[:8].float()).all(), "write before the start of out"
+    _check_canary(buf, n + 8)
+    ref, _ = oracle.attention(q, k, v, cu.tolist(), cu.tolist(), 0.09, True)
+    assert_close(out, ref, dtype=dtype, what="out at a 16-byte offset")
 
 
 def test_extreme_scores_no_overflow():
@@ -272,7 +314,9 @@ def test_decode_edges(lk, split, hq, hkv):
 
 
 @pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.float16),
-                                     (64, torch.bfloat16)])
+                                     (64, torch.bfloat16), (8, torch.bfloat16),
+                                     (40, torch.float16), (96, torch.bfloat16),
+                                     (120, torch.bfloat16)])
 def test_decode_dims(d, dtype):
     lk = [300, 1000, 65]
     _, k, v = make_qkv([1], lk, 16, 4, d, dtype, 500)
