@@ -351,21 +351,32 @@ def decode_splitkv_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     ``[B, Hq, D]``, optional ``lse`` ``[Hq, B]`` fp32) along with the inputs. Calls that overlap on
     the GPU share that array and race; keep them ordered on one stream. Raises ``MeaError`` with
     ``MEA_ERR_SCRATCH_LIMIT`` when the partials cannot fit in the array.
+
+    Nothing is copied or converted here either (a copy would allocate device memory): every
+    tensor, ``cu_seqlens_k`` and ``alibi_slopes`` included, must already be contiguous, of the
+    documented dtype and on q's GPU, otherwise ``MeaError`` is raised.
     """
     if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape or k.shape[2] != q.shape[2]:
         raise MeaError(_lib.MEA_ERR_SHAPE, "q [B, Hq, D], k/v [T_k, Hkv, D]")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise MeaError(_lib.MEA_ERR_DTYPE, "q, k and v must share one dtype")
     if not q.is_cuda:
         raise MeaError(_lib.MEA_ERR_DEVICE, "tensors must live on the GPU")
-    _on_device(q.device, k=k, v=v)
-    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    _on_device(q.device, k=k, v=v, cu_seqlens_k=cu_seqlens_k, alibi_slopes=alibi_slopes)
+    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens_k", cu_seqlens_k),
+                    ("alibi_slopes", alibi_slopes)):
+        if t is not None and not t.is_contiguous():
+            raise MeaError(_lib.MEA_ERR_SHAPE, f"{name} must be contiguous (no copy is made)")
     b, hq, d = q.shape
     tk, hkv, _ = k.shape
-    cu_seqlens_k = _check_cu("cu_seqlens_k", cu_seqlens_k, b + 1, q.device)
+    _check_cu("cu_seqlens_k", cu_seqlens_k, b + 1, q.device)
     _check_buffer("out", out, (b, hq, d), q.dtype, q.device)
     if lse is not None:
         _check_buffer("lse", lse, (hq, b), torch.float32, q.device)
-    if alibi_slopes is not None:
-        alibi_slopes = alibi_slopes.to(device=q.device, dtype=torch.float32).contiguous()
+    if alibi_slopes is not None and (alibi_slopes.dtype != torch.float32
+                                     or tuple(alibi_slopes.shape) != (hq,)):
+        raise MeaError(_lib.MEA_ERR_SHAPE,
+                       f"alibi_slopes must be a float32 [{hq}] tensor (no conversion is made)")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     rc = _lib.load().mea_decode_splitkv_noalloc(
