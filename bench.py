@@ -39,9 +39,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--part", default="all", choices=["all", "fwd", "decode", "bwd"],
+    ap.add_argument("--part", default="all", choices=["all", "fwd", "decode", "bwd", "long"],
                     help="all = the timed step (forward + decode) plus the backward measured "
-                         "on its own; bwd = the backward alone")
+                         "on its own; bwd = the backward alone; long = the 16384-token "
+                         "prefill alone (for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-paged", dest="paged", action="store_false",
                     help="skip the paged-cache decode measurement")
@@ -297,6 +298,7 @@ def run_ours(args, world, rank, local):
     do_fwd = args.part in ("all", "fwd")
     do_dec = args.part in ("all", "decode")
     do_bwd = args.part in ("all", "bwd")
+    do_long = args.part == "long" or (do_fwd and args.long)
 
     w2, w4 = workload(2), workload(4)
     g = torch.Generator(device=dev)
@@ -513,13 +515,12 @@ def run_ours(args, world, rank, local):
                    "roofline": {"bound": "tensor", "achieved": f8tf, "peak": peak8,
                                 "unit": "TFLOP/s", "frac": f8tf / peak8,
                                 "traffic": traffic_for("mea_fwd_sm100_kernel_e4m3"),
-                                "peak_kind": "dense fp8 = measured bf16 burst x 2 (nominal "
-                                             f"4.5 / 2.25 PFLOP/s), {peak_src}",
+                                "peak_kind": "fp8 = bf16 burst x 2 (nominal ratio)",
                                 "kernel": "mea_fwd_sm100_kernel<…, e4m3>"}}
 
     # ---- long-context causal prefill (16384 tokens, GQA 64/8, no ALiBi), timed on its own
     long_obj = None
-    if do_fwd and args.long:
+    if do_long:
         w3 = workload(3)
         g.manual_seed(w3.seed)
         t3 = w3.seqlens_q[0]
@@ -555,7 +556,7 @@ def run_ours(args, world, rank, local):
                     "unit": "TFLOP/s", "ms_per_call": l3ms,
                     "roofline": {"bound": "tensor", "achieved": l3tf, "peak": peak3,
                                  "unit": "TFLOP/s", "frac": l3tf / peak3, "traffic": None,
-                                 "peak_kind": f"dense bf16 burst, {peak_src}",
+                                 "peak_kind": "bf16 burst",
                                  "kernel": "mea_fwd_sm100_kernel<128, bf16, causal>",
                                  "flops_per_launch": flops3}}
         del q3, k3, v3, out3, lse3
@@ -585,9 +586,8 @@ def run_ours(args, world, rank, local):
                                   "frac": pgbs / hbm,
                                   "traffic": traffic_for("mea_decode_split_kernel_paged")
                                   if pbs == 16 else None,
-                                  "peak_kind": f"HBM copy bandwidth, {peak_src}",
-                                  "kernel": "mea_decode_split_kernel<paged> + "
-                                            "mea_lse_merge_kernel",
+                                  "peak_kind": "HBM copy",
+                                  "kernel": "decode_split<paged> + lse_merge",
                                   "bytes_per_call": dbytes}}
 
     # ---- backward on the packed prefill workload, timed on its own (not part of the step)
@@ -642,12 +642,20 @@ def run_ours(args, world, rank, local):
                    "roofline": {"bound": "tensor", "achieved": btf, "peak": peak,
                                 "unit": "TFLOP/s", "frac": btf / peak,
                                 "traffic": traffic_for("mea_backward_call"),
-                                "peak_kind": f"dense bf16 burst, {peak_src}",
-                                "kernel": "mea_bwd_pre_kernel + mea_bwd_dkdv_kernel + "
-                                          "mea_bwd_dq_kernel"},
+                                "peak_kind": "bf16 burst",
+                                "kernel": "bwd_pre + bwd_dkdv_tc + bwd_dq_tc"},
                    "memory": mem_obj}
 
     if rank != 0:
+        return 0
+    if args.part == "long":
+        line = {"metric": long_obj["metric"], "value": long_obj["value"], "unit": "TFLOP/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": long_obj["ms_per_call"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "causal prefill, 16384 tokens, GQA 64/8, D=128, bf16"},
+                "roofline": long_obj["roofline"], "gpu_launches": args.steps}
+        print(json.dumps(_compact(line)))
         return 0
 
     line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -674,25 +682,16 @@ def run_ours(args, world, rank, local):
                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                                 "frac": gbs / hbm,
                                 "traffic": traffic_for("mea_decode_split_kernel"),
-                                "peak_kind": f"HBM copy bandwidth, {peak_src}",
+                                "peak_kind": f"HBM copy, {peak_src}",
                                 "kernel": "mea_decode_split_kernel + mea_lse_merge_kernel",
                                 "bytes_per_call": dbytes}}
-        line["decode"] = dec_obj
         if not do_fwd:
             line.update({"value": dec_obj["value"], "unit": "GB/s",
                          "roofline": dec_obj["roofline"]})
-    if fp8_obj is not None:
-        line["fp8_forward"] = fp8_obj
-    if long_obj is not None:
-        line["long_prefill"] = long_obj
-    if paged_obj is not None:
-        line["paged_decode"] = paged_obj
-    if bwd_obj is not None:
-        line["backward"] = bwd_obj
-        if not do_fwd and not do_dec:
-            line.update({"value": bwd_obj["value"], "unit": "TFLOP/s",
-                         "roofline": bwd_obj["roofline"], "ms_per_step": bwd_obj["ms_per_call"]})
-            line["metric"] = bwd_obj["metric"]
+    if bwd_obj is not None and not do_fwd and not do_dec:
+        line.update({"value": bwd_obj["value"], "unit": "TFLOP/s",
+                     "roofline": bwd_obj["roofline"], "ms_per_step": bwd_obj["ms_per_call"]})
+        line["metric"] = bwd_obj["metric"]
     line["clocks"] = clk
     line["gpu_launches"] = launches_per_step * args.steps
     if e2e is not None:
@@ -702,8 +701,28 @@ def run_ours(args, world, rank, local):
         dt = time_oracle(sample)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
                                 "kind": "oracle", "sample": desc, "seconds": dt}
-    print(json.dumps(line))
+    # The extra measurements come last, the decode (the step's second metric) at the very end,
+    # so that a reader keeping only the tail of the line still has it.
+    for key, obj in (("fp8_forward", fp8_obj), ("paged_decode", paged_obj),
+                     ("backward", bwd_obj), ("long_prefill", long_obj)):
+        if obj is not None:
+            line[key] = obj
+    if do_dec:
+        line["decode"] = dec_obj
+    print(json.dumps(_compact(line)))
     return 0
+
+
+def _compact(obj):
+    """Floats rounded to 5 significant digits (the line stays short; timings are not that
+    precise anyway)."""
+    if isinstance(obj, float):
+        return float(f"{obj:.5g}") if math.isfinite(obj) else obj
+    if isinstance(obj, dict):
+        return {k: _compact(v) for k, v in obj.items()}
+    if isinstance(obj, list):
+        return [_compact(v) for v in obj]
+    return obj
 
 
 def main():

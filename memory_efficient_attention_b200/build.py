@@ -2,6 +2,7 @@
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -9,6 +10,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmea.so")
+STAMP = LIB + ".sha256"  # hash of the sources and flags libmea.so was built from
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [
@@ -30,11 +32,24 @@ def sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+def source_hash() -> str:
+    """SHA-256 over the kernel sources, the public header and the compiler flags."""
+    h = hashlib.sha256(" ".join(NVCC_FLAGS).encode())
+    for path in sources():
+        h.update(os.path.relpath(path, os.path.dirname(HERE)).encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    """True when libmea.so exists and was built from exactly the current sources (a stamp file
+    beside the library holds their hash; modification times are not trusted, since a copied
+    tree can carry a newer library built from other sources)."""
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(s) <= t for s in sources())
+    with open(STAMP) as f:
+        return f.read().strip() == source_hash()
 
 
 def build_library(force: bool = False, verbose: bool = False) -> str:
@@ -52,6 +67,8 @@ def build_library(force: bool = False, verbose: bool = False) -> str:
     if verbose:
         print(res.stderr)
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(source_hash() + "\n")
     return LIB
 
 
