@@ -39,10 +39,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--part", default="all", choices=["all", "fwd", "decode", "bwd", "long"],
+    ap.add_argument("--part", default="all",
+                    choices=["all", "fwd", "decode", "bwd", "long", "d256"],
                     help="all = the timed step (forward + decode) plus the backward measured "
-                         "on its own; bwd = the backward alone; long = the 16384-token "
-                         "prefill alone (for profiling)")
+                         "on its own; bwd = the backward alone; long / d256 = the "
+                         "16384-token prefill at head dim 128 / 256 alone (for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-paged", dest="paged", action="store_false",
                     help="skip the paged-cache decode measurement")
@@ -50,6 +51,8 @@ def parse():
                     help="skip the FP8 forward measurement")
     ap.add_argument("--no-long", dest="long", action="store_false",
                     help="skip the long-context (16384-token) prefill measurement")
+    ap.add_argument("--no-d256", dest="d256", action="store_false",
+                    help="skip the head-dim-256 long prefill measurement")
     ap.add_argument("--paged-block-size", type=int, default=16,
                     help="slots per cache block of the paged decode measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -299,6 +302,7 @@ def run_ours(args, world, rank, local):
     do_dec = args.part in ("all", "decode")
     do_bwd = args.part in ("all", "bwd")
     do_long = args.part == "long" or (do_fwd and args.long)
+    do_d256 = args.part == "d256" or (do_fwd and args.d256)
 
     w2, w4 = workload(2), workload(4)
     g = torch.Generator(device=dev)
@@ -561,6 +565,51 @@ def run_ours(args, world, rank, local):
                                  "flops_per_launch": flops3}}
         del q3, k3, v3, out3, lse3
 
+    # ---- the same long prefill at head dim 256 (the 256-wide kernel), timed on its own
+    d256_obj = None
+    if do_d256:
+        w3 = workload(3)
+        g.manual_seed(w3.seed + 256)
+        t3 = w3.seqlens_q[0]
+        q5 = torch.randn((t3, 64, 256), generator=g, device=dev, dtype=torch.float32).bfloat16()
+        k5 = torch.randn((t3, 8, 256), generator=g, device=dev, dtype=torch.float32).bfloat16()
+        v5 = torch.randn((t3, 8, 256), generator=g, device=dev, dtype=torch.float32).bfloat16()
+        cu5 = cu_seqlens(w3.seqlens_q).to(dev)
+        out5 = torch.empty_like(q5)
+        lse5 = torch.empty((64, t3), dtype=torch.float32, device=dev)
+        flops5 = fwd_flops(w3.seqlens_q, 64, 256)
+
+        def fwd5():
+            mea.attention_packed(q5, k5, v5, cu5, cu5, t3, causal=True, scale=1.0 / 16,
+                                 out=out5, lse=lse5)
+        for _ in range(args.warmup):
+            fwd5()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n5 = max(1, args.steps // 4)
+        a.record(stream)
+        for _ in range(n5):
+            fwd5()
+        b.record(stream)
+        barrier(world)
+        d5ms = dist_max(a.elapsed_time(b), world) / n5
+        code = mea.device_error()
+        if code:
+            raise RuntimeError(f"device error word {code:#x} during the D=256 prefill")
+        d5tf = flops5 / (d5ms * 1e-3) / 1e12
+        peak5 = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        d256_obj = {"metric": "attention fwd TFLOP/s (causal prefill, 16384 tokens, GQA 64/8, "
+                              "D=256, bf16)",
+                    "value": aggregate_throughput(flops5, world, d5ms) / 1e12,
+                    "unit": "TFLOP/s", "ms_per_call": d5ms, "calls": n5,
+                    "roofline": {"bound": "tensor", "achieved": d5tf, "peak": peak5,
+                                 "unit": "TFLOP/s", "frac": d5tf / peak5,
+                                 "traffic": traffic_for("mea_fwd256_sm100_kernel"),
+                                 "peak_kind": "bf16 burst",
+                                 "kernel": "mea_fwd256_sm100_kernel<bf16, causal>",
+                                 "flops_per_launch": flops5}}
+        del q5, k5, v5, out5, lse5
+
     # ---- paged-cache decode of the same requests, timed on its own (not part of the step)
     paged_obj = None
     if do_dec and args.paged:
@@ -648,13 +697,14 @@ def run_ours(args, world, rank, local):
 
     if rank != 0:
         return 0
-    if args.part == "long":
-        line = {"metric": long_obj["metric"], "value": long_obj["value"], "unit": "TFLOP/s",
+    if args.part in ("long", "d256"):
+        obj = long_obj if args.part == "long" else d256_obj
+        line = {"metric": obj["metric"], "value": obj["value"], "unit": "TFLOP/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": long_obj["ms_per_call"], "higher_is_better": True,
+                "ms_per_step": obj["ms_per_call"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": "causal prefill, 16384 tokens, GQA 64/8, D=128, bf16"},
-                "roofline": long_obj["roofline"], "gpu_launches": args.steps}
+                "config": {"workload": obj["metric"]}, "roofline": obj["roofline"],
+                "gpu_launches": args.steps}
         print(json.dumps(_compact(line)))
         return 0
 
@@ -704,7 +754,8 @@ def run_ours(args, world, rank, local):
     # The extra measurements come last, the decode (the step's second metric) at the very end,
     # so that a reader keeping only the tail of the line still has it.
     for key, obj in (("fp8_forward", fp8_obj), ("paged_decode", paged_obj),
-                     ("backward", bwd_obj), ("long_prefill", long_obj)):
+                     ("backward", bwd_obj), ("prefill_d256", d256_obj),
+                     ("long_prefill", long_obj)):
         if obj is not None:
             line[key] = obj
     if do_dec:

@@ -32,6 +32,7 @@ struct BwdParams {
   int total_k;
   int hq;
   int hkv;
+  int dh;               // head dim of the rows (<= D; the TMA zero-fills the columns past it)
   int R;                // query heads per KV head
   float scale;
   float c1;             // scale * log2(e)
@@ -44,13 +45,15 @@ __global__ void __launch_bounds__(128) mea_bwd_pre_kernel(const BwdParams p) {
   const int lane = threadIdx.x & 31;
   if (row >= static_cast<long long>(p.total_q) * p.hq) return;
   const int t = static_cast<int>(row / p.hq), h = static_cast<int>(row % p.hq);
-  constexpr int E = D / 32;  // elements per lane
-  const size_t base = (static_cast<size_t>(t) * p.hq + h) * D + lane * E;
+  // lane takes the element pairs 2*lane + 64*i of the row's dh (even) elements
+  const size_t base = (static_cast<size_t>(t) * p.hq + h) * p.dh;
   const uint16_t* o = reinterpret_cast<const uint16_t*>(p.out) + base;
   const uint16_t* g = reinterpret_cast<const uint16_t*>(p.dout) + base;
   float acc = 0.f;
 #pragma unroll
-  for (int e = 0; e < E; e += 2) {
+  for (int i = 0; i < (D + 63) / 64; ++i) {
+    const int e = 64 * i + 2 * lane;
+    if (e >= p.dh) break;
     const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + e);
     const uint32_t gv = *reinterpret_cast<const uint32_t*>(g + e);
     float o0, o1, g0, g1;

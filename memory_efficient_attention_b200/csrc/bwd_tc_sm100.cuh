@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       tc_fence_after();
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const bool any = n_iter > 0;
-      const size_t o = (static_cast<size_t>(k0 + key) * p.hkv + g) * D;
+      const size_t o = (static_cast<size_t>(k0 + key) * p.hkv + g) * p.dh;
       // the first half of the groups writes dV, the second half scale * dK, each group its
       // share of the D columns
       constexpr int HALF = C::NWG / 2 > 0 ? C::NWG / 2 : 1;
@@ -306,7 +306,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
           uint4* dp4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
           for (int u = 0; u < 4; ++u)
-            dp4[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
+            if (c * 32 + u * 8 < p.dh)
+              dp4[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
         }
       }
     }
@@ -520,7 +521,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       tc_fence_after();
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const bool any = n_jt > 0;
-      const size_t o = (static_cast<size_t>(q0 + row) * p.hq + h) * D;
+      const size_t o = (static_cast<size_t>(q0 + row) * p.hq + h) * p.dh;
       // group w writes its share of the D columns of dQ (groups past D/32 write none)
       constexpr int CHQ = (D / 32) / C::NWG > 0 ? (D / 32) / C::NWG : 1;
 #pragma unroll 1
@@ -538,7 +539,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
           uint4* dqp = reinterpret_cast<uint4*>(reinterpret_cast<OutT*>(p.dq) + o + c * 32);
 #pragma unroll
           for (int u = 0; u < 4; ++u)
-            dqp[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
+            if (c * 32 + u * 8 < p.dh)
+              dqp[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
         }
       }
     }

@@ -54,13 +54,16 @@ struct DecCfg {
   static constexpr uint32_t ATOM_BYTES = BK * 128;    // 64 keys x 128 B
   static constexpr uint32_t KT_BYTES = BK * D * 2;    // one K (or V) tile
   static constexpr uint32_t STAGE_BYTES = 2 * KT_BYTES;
-  static constexpr int NS = (D == 128) ? 5 : 8;
+  static constexpr int NS = (D == 256) ? 3 : (D == 128) ? 5 : 8;
+  // The four warps' partial O rows are merged through shared memory MC columns at a time.
+  static constexpr int MC = D < 128 ? D : 128;
   static constexpr uint32_t SMEM_RING = 0;
-  static constexpr uint32_t SMEM_MERGE = NS * STAGE_BYTES;            // 4 warps x 16 rows x D
-  static constexpr uint32_t MERGE_O_BYTES = 4 * 16 * D * 4;
+  static constexpr uint32_t SMEM_MERGE = NS * STAGE_BYTES;            // 4 warps x 16 rows x MC
+  static constexpr uint32_t MERGE_O_BYTES = 4 * 16 * MC * 4;
   static constexpr uint32_t SMEM_ML = SMEM_MERGE + MERGE_O_BYTES;     // 4 warps x 16 x (m, l)
   static constexpr uint32_t SMEM_BAR = SMEM_ML + 4 * 16 * 2 * 4;
   static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
+  static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
   static constexpr int THREADS = 160;
 };
 
@@ -244,7 +247,7 @@ __global__ void __launch_bounds__(160, 1)
     constexpr float LN2 = 0.6931471805599453f;
     const int g8 = lane >> 2;  // fragment row (head) 0..7
     const int t4 = lane & 3;   // fragment column pair
-    uint32_t cnt = 0, n_done = 0;
+    uint32_t cnt = 0, n_done = 0, m_cnt = 0;
     bool ok = true;
     for (long long lin = blockIdx.x; lin < p.n_items && ok; lin += gridDim.x) {
       const int cid = static_cast<int>(lin / p.n_hb);
@@ -414,46 +417,54 @@ __global__ void __launch_bounds__(160, 1)
       l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
       l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
       l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
-      float* mo = merge_o + warp * 16 * D;
-#pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        mo[g8 * D + n * 8 + 2 * t4] = o[n][0];
-        mo[g8 * D + n * 8 + 2 * t4 + 1] = o[n][1];
-        mo[(g8 + 8) * D + n * 8 + 2 * t4] = o[n][2];
-        mo[(g8 + 8) * D + n * 8 + 2 * t4 + 1] = o[n][3];
-      }
       if (t4 == 0) {
         merge_ml[(warp * 16 + g8) * 2 + 0] = m_lo;
         merge_ml[(warp * 16 + g8) * 2 + 1] = l_lo;
         merge_ml[(warp * 16 + g8 + 8) * 2 + 0] = m_hi;
         merge_ml[(warp * 16 + g8 + 8) * 2 + 1] = l_hi;
       }
-      mbar_arrive(DBAR(B_M0));
-      ok = mbar_wait(DBAR(B_M0), n_done & 1u, abort_flag, tmo, ecode | 3);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      for (int idx = threadIdx.x; idx < p.RB * D; idx += 128) {
-        const int row = idx / D, d = idx - row * D;
-        float M = -INFINITY;
+      float* mo = merge_o + warp * 16 * C::MC;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, merge_ml[(w * 16 + row) * 2]);
-        float Lsum = 0.f, acc = 0.f;
-        if (M != -INFINITY) {
+      for (int pass = 0; pass < D / C::MC; ++pass) {
+        // this warp's columns [pass*MC, (pass+1)*MC) of its 16 rows
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const float wt = ex2_approx(merge_ml[(w * 16 + row) * 2] - M);
-            Lsum += merge_ml[(w * 16 + row) * 2 + 1] * wt;
-            acc += merge_o[(w * 16 + row) * D + d] * wt;
-          }
+        for (int nn = 0; nn < C::MC / 8; ++nn) {
+          const int n = pass * (C::MC / 8) + nn;
+          mo[g8 * C::MC + nn * 8 + 2 * t4] = o[n][0];
+          mo[g8 * C::MC + nn * 8 + 2 * t4 + 1] = o[n][1];
+          mo[(g8 + 8) * C::MC + nn * 8 + 2 * t4] = o[n][2];
+          mo[(g8 + 8) * C::MC + nn * 8 + 2 * t4 + 1] = o[n][3];
         }
-        const int head = hb * p.RB + row;
-        const size_t slot = static_cast<size_t>(cid) * p.hq + head;
-        p.ws_o[slot * D + d] = Lsum > 0.f ? acc / Lsum : 0.f;
-        if (d == 0) p.ws_lse[slot] = Lsum > 0.f ? (M + __log2f(Lsum)) * LN2 : -INFINITY;
+        mbar_arrive(DBAR(B_M0));
+        ok = mbar_wait(DBAR(B_M0), m_cnt & 1u, abort_flag, tmo, ecode | 3);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        for (int idx = threadIdx.x; idx < p.RB * C::MC; idx += 128) {
+          const int row = idx / C::MC, dc = idx - row * C::MC;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) M = fmaxf(M, merge_ml[(w * 16 + row) * 2]);
+          float Lsum = 0.f, acc = 0.f;
+          if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float wt = ex2_approx(merge_ml[(w * 16 + row) * 2] - M);
+              Lsum += merge_ml[(w * 16 + row) * 2 + 1] * wt;
+              acc += merge_o[(w * 16 + row) * C::MC + dc] * wt;
+            }
+          }
+          const int head = hb * p.RB + row;
+          const size_t slot = static_cast<size_t>(cid) * p.hq + head;
+          const int d = pass * C::MC + dc;
+          p.ws_o[slot * D + d] = Lsum > 0.f ? acc / Lsum : 0.f;
+          if (d == 0) p.ws_lse[slot] = Lsum > 0.f ? (M + __log2f(Lsum)) * LN2 : -INFINITY;
+        }
+        mbar_arrive(DBAR(B_M1));
+        ok = mbar_wait(DBAR(B_M1), m_cnt & 1u, abort_flag, tmo, ecode | 4);
+        ok = __all_sync(0xffffffffu, ok);
+        ++m_cnt;
+        if (!ok) break;
       }
-      mbar_arrive(DBAR(B_M1));
-      ok = mbar_wait(DBAR(B_M1), n_done & 1u, abort_flag, tmo, ecode | 4);
-      ok = __all_sync(0xffffffffu, ok);
       ++n_done;
     }
   }

@@ -15,6 +15,7 @@
 #include "bwd_sm100.cuh"
 #include "bwd_tc_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "fwd256_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "ptx.cuh"
 
@@ -143,8 +144,9 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // Head dims of the forward: a multiple of 8 from 8 to 128 for 16-bit inputs (16-byte rows), a
 // multiple of 16 from 16 to 128 for e4m3 inputs.
+// Head dims from 136 to 256 (16-bit only) run in the 256-wide kernel.
 bool fwd_head_dim_ok(int d, bool e8) {
-  return e8 ? (d >= 16 && d <= 128 && d % 16 == 0) : (d >= 8 && d <= 128 && d % 8 == 0);
+  return e8 ? (d >= 16 && d <= 128 && d % 16 == 0) : (d >= 8 && d <= 256 && d % 8 == 0);
 }
 
 int largest_pow2_divisor(int x, int cap) {
@@ -202,6 +204,27 @@ int launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
 
+template <bool BF16, bool CAUSAL, bool ALIBI>
+int launch_fwd256_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    const mea::FwdParams& p, int grid, cudaStream_t stream) {
+  constexpr auto kern = mea::mea_fwd256_sm100_kernel<BF16, CAUSAL, ALIBI>;
+  constexpr uint32_t smem = mea::Fwd256Cfg::SMEM_TOTAL;
+  if (smem_attr_once<kern>(smem) != cudaSuccess) return MEA_ERR_CUDA;
+  clear_stale_launch_error();
+  kern<<<grid, mea::Fwd256Cfg::THREADS, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+template <bool BF16>
+int launch_fwd256_d(bool causal, bool alibi, const CUtensorMap& tq, const CUtensorMap& tk,
+                    const CUtensorMap& tv, const mea::FwdParams& p, int grid, cudaStream_t s) {
+  if (causal)
+    return alibi ? launch_fwd256_t<BF16, true, true>(tq, tk, tv, p, grid, s)
+                 : launch_fwd256_t<BF16, true, false>(tq, tk, tv, p, grid, s);
+  return alibi ? launch_fwd256_t<BF16, false, true>(tq, tk, tv, p, grid, s)
+               : launch_fwd256_t<BF16, false, false>(tq, tk, tv, p, grid, s);
+}
+
 template <int D, bool BF16, bool E8 = false>
 int launch_fwd_d(bool causal, bool alibi, const CUtensorMap& tq, const CUtensorMap& tk,
                  const CUtensorMap& tv, const CUtensorMap& to, const mea::FwdParams& p, int grid,
@@ -211,6 +234,17 @@ int launch_fwd_d(bool causal, bool alibi, const CUtensorMap& tq, const CUtensorM
                  : launch_fwd_t<D, BF16, true, false, E8>(tq, tk, tv, to, p, grid, s);
   return alibi ? launch_fwd_t<D, BF16, false, true, E8>(tq, tk, tv, to, p, grid, s)
                : launch_fwd_t<D, BF16, false, false, E8>(tq, tk, tv, to, p, grid, s);
+}
+
+
+// 3-D / 4-D maps through the cache (same arguments as the uncached encoders).
+bool encode_3d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  const MapKey k{base, dtype, 3, {d0, d1, d2, 0}, {b0, b1, b2, 0}};
+  if (map_lookup(k, map)) return true;
+  if (!encode_3d_uncached(map, base, dtype, d0, d1, d2, b0, b1, b2)) return false;
+  map_insert(k, *map);
+  return true;
 }
 
 // 4-D tiled map over a paged cache [d3 blocks, d2 slots, d1 heads, d0] of 16-bit elements.
@@ -229,16 +263,6 @@ bool encode_4d_uncached(CUtensorMap* map, const void* base, int dtype, uint64_t 
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
-}
-
-// 3-D / 4-D maps through the cache (same arguments as the uncached encoders).
-bool encode_3d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
-               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
-  const MapKey k{base, dtype, 3, {d0, d1, d2, 0}, {b0, b1, b2, 0}};
-  if (map_lookup(k, map)) return true;
-  if (!encode_3d_uncached(map, base, dtype, d0, d1, d2, b0, b1, b2)) return false;
-  map_insert(k, *map);
-  return true;
 }
 
 bool encode_4d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint64_t d1,
@@ -335,9 +359,9 @@ struct DecLayout {
   size_t o_bytes = 0, lse_off = 0, total = 0;
 };
 
-// Head dims of the decode: a multiple of 8 from 8 to 128; the kernels run 64 or 128 wide.
-bool dec_head_dim_ok(int d) { return d >= 8 && d <= 128 && d % 8 == 0; }
-int padded_head_dim(int d) { return d <= 64 ? 64 : 128; }
+// Head dims of the decode: a multiple of 8 from 8 to 256; the kernels run 64, 128 or 256 wide.
+bool dec_head_dim_ok(int d) { return d >= 8 && d <= 256 && d % 8 == 0; }
+int padded_head_dim(int d) { return d <= 64 ? 64 : d <= 128 ? 128 : 256; }
 
 bool dec_layout(int n_seqs, int total_k, int hq, int hkv, int d, int split_keys, int sms,
                 DecLayout& L) {
@@ -479,7 +503,8 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, float* 
   p.R = R;
   p.n_hb = n_heads_q / P;
   p.tok_per_tile = 128 / P;
-  p.subtiles = 2;
+  const bool wide = head_dim > 128;  // one 128-row sub-tile per work item
+  p.subtiles = wide ? 1 : 2;
   p.c1 = scale * qk_descale * 1.4426950408889634f;
   p.o_scale = v_descale;
   p.timeout_ns = g_timeout_ns.load();
@@ -499,13 +524,17 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, float* 
     return MEA_ERR_CUDA;
   // Every CTA walks the live items of the whole problem; max_seqlen_q only bounds how many
   // can exist, so a grid wider than that would leave CTAs idle.
-  const long long pairs_max = (static_cast<long long>(max_seqlen_q) + 2 * p.tok_per_tile - 1) /
-                              (2 * p.tok_per_tile);
+  const int tok_per_item = p.subtiles * p.tok_per_tile;
+  const long long pairs_max =
+      (static_cast<long long>(max_seqlen_q) + tok_per_item - 1) / tok_per_item;
   const long long items_max = pairs_max * n_seqs * p.n_hb;
   const int grid = static_cast<int>(items_max < di.sms ? (items_max > 0 ? items_max : 1) : di.sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool causal = mask_kind == MEA_MASK_CAUSAL;
   const bool alibi = alibi_slopes != nullptr;
+  if (wide)
+    return dtype == MEA_BF16 ? launch_fwd256_d<true>(causal, alibi, tq, tk, tv, p, grid, s)
+                             : launch_fwd256_d<false>(causal, alibi, tq, tk, tv, p, grid, s);
   if (e8)
     return dtype == MEA_BF16
                ? launch_fwd_d<128, true, true>(causal, alibi, tq, tk, tv, to, p, grid, s)
@@ -589,7 +618,7 @@ int mea_backward(const void* q, const void* k, const void* v, const void* out, c
       max_seqlen_k < 0 || max_seqlen_q > total_q || max_seqlen_k > total_k)
     return MEA_ERR_SHAPE;
   if (n_heads_q < 1 || n_heads_kv < 1 || n_heads_q % n_heads_kv != 0) return MEA_ERR_HEADS;
-  if (head_dim != 64 && head_dim != 128) return MEA_ERR_HEAD_DIM;
+  if (!dec_head_dim_ok(head_dim) || head_dim > 128) return MEA_ERR_HEAD_DIM;
   if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_DTYPE;
   if (mask_kind != MEA_MASK_NONE && mask_kind != MEA_MASK_CAUSAL) return MEA_ERR_MASK;
   if (!std::isfinite(scale)) return MEA_ERR_SCALE;
@@ -624,6 +653,7 @@ int mea_backward(const void* q, const void* k, const void* v, const void* out, c
   p.total_k = total_k;
   p.hq = n_heads_q;
   p.hkv = n_heads_kv;
+  p.dh = head_dim;
   p.R = n_heads_q / n_heads_kv;
   p.scale = scale;
   p.c1 = scale * 1.4426950408889634f;
@@ -638,7 +668,7 @@ int mea_backward(const void* q, const void* k, const void* v, const void* out, c
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool causal = mask_kind == MEA_MASK_CAUSAL;
   const bool alibi = alibi_slopes != nullptr;
-  if (head_dim == 128)
+  if (head_dim > 64)
     return dtype == MEA_BF16
                ? launch_bwd_d<128, true>(causal, alibi, m, p, max_seqlen_q, max_seqlen_k, s)
                : launch_bwd_d<128, false>(causal, alibi, m, p, max_seqlen_q, max_seqlen_k, s);
@@ -737,6 +767,9 @@ int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, f
   const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool alibi = alibi_slopes != nullptr;
+  if (head_dim > 128)
+    return dtype == MEA_BF16 ? launch_dec_d<256, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+                             : launch_dec_d<256, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
   if (head_dim > 64)
     return dtype == MEA_BF16 ? launch_dec_d<128, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
                              : launch_dec_d<128, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
@@ -812,6 +845,10 @@ int mea_decode_paged(const void* q, const void* k_cache, const void* v_cache,
   const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool alibi = alibi_slopes != nullptr;
+  if (head_dim > 128)
+    return dtype == MEA_BF16
+               ? launch_dec_d<256, true, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+               : launch_dec_d<256, false, true>(alibi, tk, tv, p, grid, n_heads_kv, s);
   if (head_dim > 64)
     return dtype == MEA_BF16
                ? launch_dec_d<128, true, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
@@ -892,6 +929,9 @@ int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void
   const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool alibi = alibi_slopes != nullptr;
+  if (head_dim > 128)
+    return dtype == MEA_BF16 ? launch_dec_d<256, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
+                             : launch_dec_d<256, false>(alibi, tk, tv, p, grid, n_heads_kv, s);
   if (head_dim > 64)
     return dtype == MEA_BF16 ? launch_dec_d<128, true>(alibi, tk, tv, p, grid, n_heads_kv, s)
                              : launch_dec_d<128, false>(alibi, tk, tv, p, grid, n_heads_kv, s);

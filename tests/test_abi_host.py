@@ -68,7 +68,7 @@ def fwd(lib, **kw):
     (dict(hq=6, hkv=4), _lib.MEA_ERR_HEADS),
     (dict(hkv=0), _lib.MEA_ERR_HEADS),
     (dict(d=100), _lib.MEA_ERR_HEAD_DIM),
-    (dict(d=136), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=264), _lib.MEA_ERR_HEAD_DIM),
     (dict(d=0), _lib.MEA_ERR_HEAD_DIM),
     (dict(dtype=2), _lib.MEA_ERR_DTYPE),
     (dict(mask=2), _lib.MEA_ERR_MASK),
@@ -101,7 +101,7 @@ def dec(lib, **kw):
     (dict(split=100), _lib.MEA_ERR_SHAPE),
     (dict(hq=12, hkv=8), _lib.MEA_ERR_HEADS),
     (dict(d=36), _lib.MEA_ERR_HEAD_DIM),
-    (dict(d=256), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=264), _lib.MEA_ERR_HEAD_DIM),
     (dict(dtype=-1), _lib.MEA_ERR_DTYPE),
     (dict(mask=3), _lib.MEA_ERR_MASK),
     (dict(v=A + 4), _lib.MEA_ERR_ALIGN),
@@ -149,7 +149,8 @@ def bwd(lib, **kw):
     (dict(max_q=101), _lib.MEA_ERR_SHAPE),
     (dict(max_k=121), _lib.MEA_ERR_SHAPE),
     (dict(hq=6, hkv=4), _lib.MEA_ERR_HEADS),
-    (dict(d=96), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=100), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=256), _lib.MEA_ERR_HEAD_DIM),
     (dict(dtype=5), _lib.MEA_ERR_DTYPE),
     (dict(mask=-1), _lib.MEA_ERR_MASK),
     (dict(scale=float("nan")), _lib.MEA_ERR_SCALE),
@@ -196,7 +197,7 @@ def paged(lib, **kw):
     (dict(split=100), _lib.MEA_ERR_SHAPE),
     (dict(hq=12, hkv=8), _lib.MEA_ERR_HEADS),
     (dict(d=84), _lib.MEA_ERR_HEAD_DIM),
-    (dict(d=192), _lib.MEA_ERR_HEAD_DIM),
+    (dict(d=512), _lib.MEA_ERR_HEAD_DIM),
     (dict(dtype=7), _lib.MEA_ERR_DTYPE),
     (dict(table=A + 2), _lib.MEA_ERR_ALIGN),
     (dict(vc=A + 8), _lib.MEA_ERR_ALIGN),

@@ -132,6 +132,12 @@ def test_backward_dtypes_dims_masks(d, dtype, causal, alibi):
     _check([190, 65], [190, 65], 4, 2, d, dtype, causal, alibi, 0.11, 950)
 
 
+@pytest.mark.parametrize("d", [8, 32, 40, 72, 96, 120])
+def test_backward_other_head_dims(d):
+    # multiples of 8 up to 128: the 64- or 128-wide kernels with zero-filled columns
+    _check([190, 65], [190, 65], 4, 2, d, torch.bfloat16, True, True, 1 / math.sqrt(d), 955 + d)
+
+
 @pytest.mark.parametrize("lens", [[63], [64], [65], [128], [129], [1], [2, 3]])
 def test_backward_tile_edges(lens):
     _check(lens, lens, 4, 2, 128, torch.bfloat16, True, False, 0.09, 960 + sum(lens))

@@ -89,7 +89,7 @@ def test_paged_decode_block_sizes(bs):
            1 / math.sqrt(128), 1100 + bs)
 
 
-@pytest.mark.parametrize("d", [40, 64, 96, 128])
+@pytest.mark.parametrize("d", [40, 64, 96, 128, 256])
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("alibi", [False, True])
 def test_paged_decode_dtypes_dims_alibi(d, dtype, alibi):

@@ -181,6 +181,41 @@ def test_dtypes_dims_masks(d, dtype, causal, alibi):
     check_packed(lens, lens, 8, 2, d, dtype, causal, alibi, 1.0 / math.sqrt(d), 300 + d)
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("causal,alibi", [(False, False), (True, False), (True, True),
+                                          (False, True)])
+def test_head_dim_256(dtype, causal, alibi):
+    # the 256-wide kernel: one 128-row tile per item, S double-buffered in tensor memory
+    lens = [190, 1, 64, 385, 129]
+    check_packed(lens, lens, 8, 2, 256, dtype, causal, alibi, 1.0 / 16, 360)
+
+
+@pytest.mark.parametrize("hq,hkv", [(1, 1), (4, 1), (6, 2), (32, 2), (128, 1)])
+def test_head_dim_256_gqa_and_edges(hq, hkv):
+    lens = [1, 127, 128, 129, 300, 5]
+    check_packed(lens, lens, hq, hkv, 256, torch.bfloat16, True, hq <= 32, 0.07, 370 + hq)
+
+
+def test_head_dim_256_lq_ne_lk_and_empty():
+    lq = [5, 130, 40, 0, 17]
+    lk = [300, 140, 10, 9, 0]
+    for causal in (False, True):
+        check_packed(lq, lk, 8, 4, 256, torch.bfloat16, causal, True, 0.06, 380)
+
+
+@pytest.mark.parametrize("d", [136, 192, 200, 248])
+def test_head_dims_between_128_and_256(d):
+    lens = [130, 7, 300]
+    check_packed(lens, lens, 8, 2, d, torch.bfloat16, True, True, 1.0 / math.sqrt(d), 390 + d)
+
+
+def test_head_dim_256_long_segments_many_items():
+    # several thousand keys per row: long runs of the S double buffer, rescales of O
+    lens = [3000, 2100, 700]
+    check_packed(lens, lens, 16, 4, 256, torch.bfloat16, True, True, 0.0625, 395)
+    check_packed(lens, lens, 16, 4, 256, torch.float16, True, False, 0.125, 396)
+
+
 @pytest.mark.parametrize("d", [8, 16, 40, 72, 80, 120])
 def test_other_head_dims(d):
     # any multiple of 8 up to 128: the 64- or 128-wide kernel with zero-filled columns
@@ -316,7 +351,8 @@ def test_decode_edges(lk, split, hq, hkv):
 @pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.float16),
                                      (64, torch.bfloat16), (8, torch.bfloat16),
                                      (40, torch.float16), (96, torch.bfloat16),
-                                     (120, torch.bfloat16)])
+                                     (120, torch.bfloat16), (256, torch.bfloat16),
+                                     (256, torch.float16), (200, torch.bfloat16)])
 def test_decode_dims(d, dtype):
     lk = [300, 1000, 65]
     _, k, v = make_qkv([1], lk, 16, 4, d, dtype, 500)
@@ -326,6 +362,24 @@ def test_decode_dims(d, dtype):
     torch.cuda.synchronize()
     ro, rl = oracle.decode(q, k, v, cu_seqlens(lk).tolist(), 1 / math.sqrt(d))
     assert_close(out, ro, lse, rl, dtype, f"decode D{d} {dtype}")
+
+
+@pytest.mark.parametrize("hq,hkv", [(64, 8), (16, 1), (12, 2)])
+def test_decode_head_dim_256_edges(hq, hkv):
+    lk = [1, 64, 65, 0, 2000, 129]
+    _, k, v = make_qkv([1], lk, hq, hkv, 256, torch.bfloat16, 410 + hq)
+    q = make_qkv([len(lk)], [1], hq, hkv, 256, torch.bfloat16, 411 + hq)[0]
+    slopes = alibi_slope_values(hq)
+    obuf, out = _alloc_out((len(lk), hq, 256), torch.bfloat16)
+    lbuf, lse = _alloc_lse((hq, len(lk)))
+    mea.decode_splitkv(q.cuda(), k.cuda(), v.cuda(), cu_seqlens(lk).cuda(), max(lk),
+                       alibi_slopes=slopes.cuda(), scale=0.0625, split_keys=128, out=out,
+                       lse=lse)
+    torch.cuda.synchronize()
+    _check_canary(obuf, out.numel())
+    _check_canary(lbuf, lse.numel())
+    ro, rl = oracle.decode(q, k, v, cu_seqlens(lk).tolist(), 0.0625, slopes.double())
+    assert_close(out, ro, lse, rl, torch.bfloat16, f"decode D256 H{hq}/{hkv}")
 
 
 def test_decode_matches_forward():
