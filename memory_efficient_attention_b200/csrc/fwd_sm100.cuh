@@ -319,15 +319,15 @@ __device__ __forceinline__ uint32_t fp8x2_e4m3(float lo, float hi) {
 
 // p(c) = 2^(c1*x(c) + slope2*c - off) (slope2 term only with ALiBi) for the 128 columns of this
 // thread's row, packed to 16-bit pairs over the first 64 TMEM columns at t_s (E8: to e4m3
-// quadruples over the first 32 columns). Returns the row sum of p in fp32 and, in emax, the
-// largest exponent seen.
+// quadruples over the first 32 columns). Returns the row sum of p in fp32. (No running maximum
+// is kept here: the softmax issue slots are the scarce resource, and the sum alone tells
+// whether any p exceeded the caller's bound.)
 template <bool BF16, bool ALIBI, bool E8 = false>
 __device__ __forceinline__ float exp_tile_to_tmem(const float (&x)[128], float c1, float slope2,
-                                                  float off, uint32_t t_s, float& emax) {
+                                                  float off, uint32_t t_s) {
   const uint64_t c1x2 = f2_pack(c1, c1);
   const uint64_t inc = f2_pack(2.f * slope2, 2.f * slope2);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-  float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
   for (int c4 = 0; c4 < 4; ++c4) {
     uint64_t cb = ALIBI ? f2_pack(slope2 * static_cast<float>(c4 * 32) - off,
@@ -340,10 +340,6 @@ __device__ __forceinline__ float exp_tile_to_tmem(const float (&x)[128], float c
       float e0, e1;
       f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), c1x2, cb), e0, e1);
       if (ALIBI) cb = f2_add(cb, inc);
-      if (i & 1)
-        m1 = max3f(m1, e0, e1);
-      else
-        m0 = max3f(m0, e0, e1);
       const float p0 = ex2_approx(e0);
       const float p1 = ex2_approx(e1);
       acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
@@ -362,7 +358,6 @@ __device__ __forceinline__ float exp_tile_to_tmem(const float (&x)[128], float c
     else
       tmem_st16(t_s + c4 * 16, pk);
   }
-  emax = fmaxf(m0, m1);
   const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
   float r0, r1;
   f2_unpack(t, r0, r1);
@@ -408,8 +403,8 @@ __device__ __forceinline__ bool fwd_softmax_tile(const FwdParams& p, uint32_t t_
         if (c > limit) x[c] = -INFINITY;
     }
     // Tiles are visited diagonal-first, so once a reference maximum exists the next tile
-    // rarely exceeds it by more than 2^8: exponentiate against it straight away and take
-    // the tile maximum on the side; redo the tile in the rare case it does.
+    // rarely takes p out of range: exponentiate against it straight away and redo the tile in
+    // the rare case it does. The first tile of a row takes its maximum first.
     const bool speculate = __all_sync(0xffffffffu, m_ref != -INFINITY);
     if (!speculate) {
       const float m_tile = tile_score_max<ALIBI>(x, p.c1, slope2) + kconst;
@@ -422,21 +417,23 @@ __device__ __forceinline__ bool fwd_softmax_tile(const FwdParams& p, uint32_t t_
       }
     }
     const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-    float emax;
-    float rs =
-        exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_use - kconst, t_s, emax);
+    float rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_use - kconst, t_s);
     if (speculate) {
-      const bool over = emax > 8.0f;
+      // Every p of the tile is at most its row sum, so a sum within the bound keeps every p
+      // within the range P is packed into: 2^15 for 16-bit P (f16 holds up to 65504; bf16 has
+      // fp32's range), 2^8 for e4m3 (448). Otherwise (rare: key tiles are visited from the
+      // diagonal down) take the tile's true maximum and redo the tile against it. The bound
+      // only limits how far the reference maximum may lag; O and l stay in fp32 either way.
+      const bool over = rs > (E8 ? 256.0f : 32768.0f);
       if (__any_sync(0xffffffffu, over)) {
-        if (over) {
-          const float m_tile = emax + m_use;
+        const float m_tile = tile_score_max<ALIBI>(x, p.c1, slope2) + kconst;
+        if (m_tile > m_ref) {
           resc = true;
           alpha = ex2_approx(m_ref - m_tile);
           l *= alpha;
           m_ref = m_tile;
         }
-        rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_ref - kconst, t_s,
-                                               emax);
+        rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_ref - kconst, t_s);
       }
     }
     l += rs;
@@ -458,8 +455,7 @@ __device__ __forceinline__ bool fwd_softmax_tile(const FwdParams& p, uint32_t t_
       m_ref = m_new;
     }
     const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-    float unused;
-    l += exp_tile_to_tmem<BF16, false, E8>(x, 1.f, 0.f, m_use, t_s, unused);
+    l += exp_tile_to_tmem<BF16, false, E8>(x, 1.f, 0.f, m_use, t_s);
   }
   return resc;
 }
