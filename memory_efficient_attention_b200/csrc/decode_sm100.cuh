@@ -32,6 +32,9 @@ struct DecParams {
   int block_size;              // paged: keys per cache block (16, 32 or a multiple of 64)
   int max_blocks;              // paged: row length of block_table
   int num_blocks;              // paged: blocks in the cache (ids outside [0, num_blocks) read 0)
+  int box5;                    // paged: 1 = one 5-D box per block covers every 64-column atom
+                               // (head_dim a multiple of 64), 0 = one 4-D box per atom
+  int lay_log2;                // log2 of the rows per shared-memory layout group (see below)
   float* ws_o;        // [n_slots, hq, D]
   float* ws_lse;      // [n_slots, hq]
   int n_seqs;
@@ -46,6 +49,18 @@ struct DecParams {
   float c1;           // scale * log2(e)
   unsigned long long timeout_ns;
 };
+
+// Shared-memory layout of a K (or V) stage: groups of 2^lay_log2 key rows, each group
+// [atom][rows][128 B] with the 128-byte swizzle. Packed K/V and 4-D paged boxes use one group of
+// 64 rows ([atom][64 keys]); 5-D paged boxes land one cache block (min(block_size, 64) rows,
+// every atom) per group. Address of 16-byte chunk ch (along D) of key row kr:
+template <int D>
+__device__ __forceinline__ uint32_t dec_row_addr(uint32_t base, int kr, int ch, int lay_log2) {
+  const uint32_t lr = 1u << lay_log2;
+  return base + static_cast<uint32_t>(kr >> lay_log2) * (lr * (D / 64) * 128u) +
+         static_cast<uint32_t>(ch >> 3) * (lr * 128u) + static_cast<uint32_t>(kr & (lr - 1)) * 128u +
+         (static_cast<uint32_t>((ch & 7) ^ (kr & 7)) << 4);
+}
 
 template <int D>
 struct DecCfg {
@@ -176,26 +191,35 @@ __global__ void __launch_bounds__(160, 1)
         // and per (K or V, 64-column atom) for block sizes 16 and 32 (boxes of block_size rows
         // at row offsets that keep the 128-B swizzle aligned), or a 64-row slice of one block
         // for block sizes that are multiples of 64. The boxes of a stage are issued by as many
-        // lanes, each of which also reads its block id one tile ahead (at 16-slot blocks a
+        // lanes, each of which also reads its block ids ahead (at 16-slot blocks a
         // stage is 16 boxes of 2 KB, and one lane issuing them all starved the stream). Blocks
         // past the request's last one use id num_blocks, which the TMA fills with zeros.
         const int32_t* row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
         const int bs = p.block_size;
         const int per = bs >= C::BK ? 1 : C::BK / bs;
         const int nblk = min((L + bs - 1) / bs, p.max_blocks);
-        const int nbox = per * 2 * C::ATOMS;               // <= 16 boxes per stage
-        const int my_i = lane / (2 * C::ATOMS);            // block of the tile
-        const int my_v = (lane / C::ATOMS) & 1;            // K or V
-        const int my_a = lane % C::ATOMS;                  // 64-column atom
+        // 4-D: one box per (block, K or V, atom), <= 16 per stage; 5-D: one per (block, K or V)
+        const int apb = p.box5 ? 1 : C::ATOMS;             // boxes per block and tensor
+        const int nbox = per * 2 * apb;
+        const int my_i = lane / (2 * apb);                 // block of the tile
+        const int my_v = (lane / apb) & 1;                 // K or V
+        const int my_a = lane % apb;                       // 64-column atom (4-D)
         const bool issuer = lane < nbox;
         auto block_id = [&](int t) {
           const int j = (key0 + t * C::BK + my_i * bs) / bs;
           return (issuer && t < n_tiles && j < nblk) ? __ldg(row + j) : p.num_blocks;
         };
-        int id_next = block_id(0);
+        // Block ids of tiles t .. t+3: each read is in flight for three tiles before its TMA
+        // needs it (a block-table line that misses in L2 waits on HBM under a full load).
+        int id_q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) id_q[u] = block_id(u);
         for (int t = 0; t < n_tiles; ++t) {
-          const int id = id_next;
-          id_next = block_id(t + 1);
+          const int id = id_q[0];
+          id_q[0] = id_q[1];
+          id_q[1] = id_q[2];
+          id_q[2] = id_q[3];
+          id_q[3] = block_id(t + 4);
           const uint32_t s = cnt % C::NS;
           const uint32_t ph = (cnt / C::NS) & 1u;
           if (lane == 0) {
@@ -205,11 +229,16 @@ __global__ void __launch_bounds__(160, 1)
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
           if (issuer) {
-            const uint32_t dst = sbase + C::SMEM_RING + s * C::STAGE_BYTES +
-                                 my_v * C::KT_BYTES + my_a * C::ATOM_BYTES +
-                                 static_cast<uint32_t>(my_i * bs * 128);
             const int r0 = bs >= C::BK ? (key0 + t * C::BK) % bs : 0;
-            tma_load_4d(dst, my_v ? &tm_v : &tm_k, DBAR(B_F + s), my_a * 64, g, r0, id);
+            const uint32_t stg = sbase + C::SMEM_RING + s * C::STAGE_BYTES + my_v * C::KT_BYTES;
+            if (p.box5) {
+              // the block's rows for every atom: [atom][rows][128 B], one layout group
+              const uint32_t dst = stg + static_cast<uint32_t>(my_i * bs * C::ATOMS * 128);
+              tma_load_5d(dst, my_v ? &tm_v : &tm_k, DBAR(B_F + s), 0, r0, 0, g, id);
+            } else {
+              const uint32_t dst = stg + my_a * C::ATOM_BYTES + static_cast<uint32_t>(my_i * bs * 128);
+              tma_load_4d(dst, my_v ? &tm_v : &tm_k, DBAR(B_F + s), my_a * 64, g, r0, id);
+            }
           }
           ++cnt;
         }
@@ -306,7 +335,7 @@ __global__ void __launch_bounds__(160, 1)
             const int r_lo = max(valid, warp * 16), r_hi = warp * 16 + 16;
             for (int i = lane; i < (r_hi > r_lo ? (r_hi - r_lo) * (D / 8) : 0); i += 32) {
               const int rr = r_lo + i / (D / 8), ch = i % (D / 8);
-              const uint32_t addr = vst + (ch >> 3) * C::ATOM_BYTES + rr * 128 + ((ch & 7) << 4);
+              const uint32_t addr = dec_row_addr<D>(vst, rr, ch ^ (rr & 7), p.lay_log2);
               asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u)
                            : "memory");
             }
@@ -322,8 +351,9 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const int ch = 2 * kk + csel;  // 16-byte chunk along D
-            const uint32_t addr = kst + (ch >> 3) * C::ATOM_BYTES + kr * 128 +
-                                  ((((ch & 7) ^ (kr & 7))) << 4);
+            const uint32_t addr = PAGED ? dec_row_addr<D>(kst, kr, ch, p.lay_log2)
+                                        : kst + (ch >> 3) * C::ATOM_BYTES + kr * 128 +
+                                              ((((ch & 7) ^ (kr & 7))) << 4);
             uint32_t r0, r1, r2, r3;
             ldsm_x4(addr, r0, r1, r2, r3);
             mma16816<BF16>(sc[0], qa[kk], r0, r1);
@@ -397,8 +427,9 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
           for (int n = 0; n < D / 8; n += 2) {
             const int ch = n + csel;
-            const uint32_t addr = vst + (ch >> 3) * C::ATOM_BYTES + kr * 128 +
-                                  ((((ch & 7) ^ (kr & 7))) << 4);
+            const uint32_t addr = PAGED ? dec_row_addr<D>(vst, kr, ch, p.lay_log2)
+                                        : vst + (ch >> 3) * C::ATOM_BYTES + kr * 128 +
+                                              ((((ch & 7) ^ (kr & 7))) << 4);
             uint32_t r0, r1, r2, r3;
             ldsm_x4_t(addr, r0, r1, r2, r3);
             mma16816<BF16>(o[n], pa, r0, r1);

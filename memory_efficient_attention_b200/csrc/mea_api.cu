@@ -94,11 +94,11 @@ bool encode_3d_uncached(CUtensorMap* map, const void* base, int dtype, uint64_t 
 struct MapKey {
   const void* base;
   int dtype, rank;
-  uint64_t dims[4];
-  uint32_t box[4];
+  uint64_t dims[5];
+  uint32_t box[5];
   bool operator==(const MapKey& o) const {
     if (base != o.base || dtype != o.dtype || rank != o.rank) return false;
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 5; ++i)
       if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
     return true;
   }
@@ -270,6 +270,31 @@ bool encode_4d(CUtensorMap* map, const void* base, int dtype, uint64_t d0, uint6
   const MapKey k{base, dtype, 4, {d0, d1, d2, d3}, {b0, b1, b2, b3}};
   if (map_lookup(k, map)) return true;
   if (!encode_4d_uncached(map, base, dtype, d0, d1, d2, d3, b0, b1, b2, b3)) return false;
+  map_insert(k, *map);
+  return true;
+}
+
+// 5-D tiled map over a paged cache [blocks, slots, heads, head_dim] of 16-bit elements with
+// head_dim = 64 * atoms, seen as (64 columns, slot, atom, head, block): one box {64, rows, atoms,
+// 1, 1} brings `rows` slots of one head and block with every 64-column atom, landing as
+// [atom][rows][128 B] (the 128-byte swizzle per 128-byte row).
+bool encode_paged5(CUtensorMap* map, const void* base, int dtype, uint64_t head_dim,
+                   uint64_t heads, uint64_t slots, uint64_t blocks, uint32_t rows) {
+  const uint64_t atoms = head_dim / 64;
+  const MapKey k{base, dtype, 5, {64, slots, atoms, heads, blocks}, {64, rows, uint32_t(atoms), 1, 1}};
+  if (map_lookup(k, map)) return true;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[5] = {64, slots, atoms, heads, blocks};
+  cuuint64_t strides[4] = {heads * head_dim * 2, 128, head_dim * 2, slots * heads * head_dim * 2};
+  cuuint32_t box[5] = {64, rows, static_cast<cuuint32_t>(atoms), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, dtype == MEA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
   map_insert(k, *map);
   return true;
 }
@@ -837,11 +862,20 @@ int mea_decode_paged(const void* q, const void* k_cache, const void* v_cache,
 
   CUtensorMap tk, tv;
   const uint32_t rows = block_size < 64 ? static_cast<uint32_t>(block_size) : 64u;
-  if (!encode_4d(&tk, k_cache, dtype, head_dim, n_heads_kv, block_size, num_blocks, 64, 1, rows,
-                 1) ||
-      !encode_4d(&tv, v_cache, dtype, head_dim, n_heads_kv, block_size, num_blocks, 64, 1, rows,
-                 1))
+  // Head dims equal to the kernel's width (64, 128, 256) take one box per block (every atom at
+  // once); the others one box per atom, whose zero fill covers the columns past head_dim.
+  p.box5 = (head_dim == 64 || head_dim == 128 || head_dim == 256) ? 1 : 0;
+  p.lay_log2 = p.box5 ? (rows == 16 ? 4 : rows == 32 ? 5 : 6) : 6;
+  if (p.box5) {
+    if (!encode_paged5(&tk, k_cache, dtype, head_dim, n_heads_kv, block_size, num_blocks, rows) ||
+        !encode_paged5(&tv, v_cache, dtype, head_dim, n_heads_kv, block_size, num_blocks, rows))
+      return MEA_ERR_CUDA;
+  } else if (!encode_4d(&tk, k_cache, dtype, head_dim, n_heads_kv, block_size, num_blocks, 64, 1,
+                        rows, 1) ||
+             !encode_4d(&tv, v_cache, dtype, head_dim, n_heads_kv, block_size, num_blocks, 64, 1,
+                        rows, 1)) {
     return MEA_ERR_CUDA;
+  }
   const int grid = total_k > 0 ? static_cast<int>(p.n_items < di.sms ? p.n_items : di.sms) : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool alibi = alibi_slopes != nullptr;
