@@ -46,7 +46,9 @@ struct BwdTcCfg {
   static constexpr uint32_t SMEM_B = TILE_BYTES;         // V (dkdv) / dO (dq), loaded once
   static constexpr uint32_t SMEM_RING = 2 * TILE_BYTES;  // 2 stages x 2 tiles
   static constexpr uint32_t SMEM_BAR = SMEM_RING + 4 * TILE_BYTES;
-  static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
+  // 256 B per elementwise warp: the row terms of its current 32-row chunk (dK/dV kernel)
+  static constexpr uint32_t SMEM_STAGE = SMEM_BAR + 256;
+  static constexpr uint32_t SMEM_TOTAL = SMEM_STAGE + 4 * 4 * 256 + 1024;
   static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
   static constexpr int NWG = 4;                          // elementwise warpgroups
   static constexpr int CPW = 4 / NWG;                      // 32-column chunks per group
@@ -65,6 +67,118 @@ struct BwdTcCfg {
 template <bool BF16>
 __device__ __forceinline__ uint32_t bpack2(float lo, float hi) {
   return dpack2<BF16>(lo, hi);
+}
+
+__device__ __forceinline__ void lds_f4(uint32_t addr, float& a, float& b, float& c, float& d) {
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(a), "=f"(b), "=f"(c), "=f"(d)
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// Bias forms of the scores: none, causal ALiBi (the distance row + shift - key is >= 0 wherever
+// p can be non-zero, so the bias is linear in row and key), ALiBi without the causal mask
+// (|row + shift - key|).
+enum { BIAS_NONE = 0, BIAS_LINEAR = 1, BIAS_ABS = 2 };
+
+// dK/dV elementwise step for half H (rows rc0 + 16H .. +15) of a 32-row chunk of the
+// S^T / dP^T tiles and this thread's key:
+//   p_e = 2^(c1 S_e + na_e + kb),  dS_e = p_e (dP_e + nd_e),  e = 0..31 (row rc0 + e)
+// with the row terms staged by the warp in shared memory as 16 float4 {na_e, na_e+1, nd_e,
+// nd_e+1}: na_e = -(lse_e log2 e) (BIAS_LINEAR: also - slope2 e), nd_e = -delta_e. kb is this
+// thread's key term (BIAS_LINEAR: -slope2 (rc0 + shift - key)); BIAS_ABS subtracts
+// slope2 |dabs + e| per element. MASK: p_e = 0 outside e_lo <= e < e_hi. sv / dv hold the
+// half's 16 S / dP columns. Pairs of columns go through the f32x2 pipe; P and dS leave packed
+// to 16 bits as eight words each, to TMEM at t_p + 8H and t_d + 8H (the chunk's own S / dP
+// columns, already read).
+template <bool BF16, bool MASK, int BIAS, int H>
+__device__ __forceinline__ void bwd_kv_half(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
+                                            uint32_t stage, uint64_t c1x2, uint64_t kb2,
+                                            float slope2, float dabs, int e_lo, int e_hi,
+                                            uint32_t t_p, uint32_t t_d) {
+  uint32_t pp[8], pd[8];
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int j = H * 8 + jj;  // column pair of the chunk
+    float na0, na1, nd0, nd1;
+    lds_f4(stage + 16u * j, na0, na1, nd0, nd1);
+    uint64_t b2 = f2_pack(na0, na1);
+    if constexpr (BIAS == BIAS_LINEAR) b2 = f2_add(b2, kb2);
+    const uint64_t z2 =
+        f2_fma(f2_pack(__uint_as_float(sv[2 * jj]), __uint_as_float(sv[2 * jj + 1])), c1x2, b2);
+    float z0, z1;
+    f2_unpack(z2, z0, z1);
+    if constexpr (BIAS == BIAS_ABS) {
+      z0 = fmaf(-slope2, fabsf(dabs + static_cast<float>(2 * j)), z0);
+      z1 = fmaf(-slope2, fabsf(dabs + static_cast<float>(2 * j + 1)), z1);
+    }
+    float p0 = ex2_approx(z0), p1 = ex2_approx(z1);
+    if constexpr (MASK) {
+      p0 = (2 * j >= e_lo && 2 * j < e_hi) ? p0 : 0.f;
+      p1 = (2 * j + 1 >= e_lo && 2 * j + 1 < e_hi) ? p1 : 0.f;
+    }
+    const uint64_t d2 = f2_mul(
+        f2_pack(p0, p1),
+        f2_add(f2_pack(__uint_as_float(dv[2 * jj]), __uint_as_float(dv[2 * jj + 1])),
+               f2_pack(nd0, nd1)));
+    float d0, d1;
+    f2_unpack(d2, d0, d1);
+    pp[jj] = bpack2<BF16>(p0, p1);
+    pd[jj] = bpack2<BF16>(d0, d1);
+  }
+  tmem_st8(t_p + H * 8, pp);
+  tmem_st8(t_d + H * 8, pd);
+}
+
+// dQ elementwise step for one 32-key chunk of the S / dP tiles and this thread's row:
+//   p_e = 2^(c1 S_e + b + slope2 e),  dS_e = p_e (dP_e - delta),  e = 0..31 (key kc0 + e)
+// with b = -lse log2 e (BIAS_LINEAR: - slope2 (row + shift - kc0)); BIAS_ABS subtracts
+// slope2 |dabs - e| per element (dabs = row + shift - kc0). MASK: p_e = 0 for e >= e_hi. dS
+// leaves packed to 16 bits, eight words at a time, to TMEM at t_d.
+template <bool BF16, bool MASK, int BIAS>
+__device__ __forceinline__ void bwd_q_chunk(const uint32_t (&sv)[32], const uint32_t (&dv)[32],
+                                            uint64_t c1x2, float b, float slope2, float dabs,
+                                            uint64_t nd2, int e_hi, uint32_t t_d) {
+  const uint64_t b2 = f2_pack(b, b);
+  const uint64_t s2 = f2_pack(slope2, slope2);
+  const uint64_t two2 = f2_pack(2.f, 2.f);
+  uint64_t e2 = f2_pack(0.f, 1.f);  // exact small integers
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+  uint32_t pd[8];
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int j = hh * 8 + jj;
+    uint64_t t2 = b2;
+    if constexpr (BIAS == BIAS_LINEAR) {
+      t2 = f2_fma(s2, e2, b2);
+      e2 = f2_add(e2, two2);
+    }
+    const uint64_t z2 =
+        f2_fma(f2_pack(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), c1x2, t2);
+    float z0, z1;
+    f2_unpack(z2, z0, z1);
+    if constexpr (BIAS == BIAS_ABS) {
+      z0 = fmaf(-slope2, fabsf(dabs - static_cast<float>(2 * j)), z0);
+      z1 = fmaf(-slope2, fabsf(dabs - static_cast<float>(2 * j + 1)), z1);
+    }
+    float p0 = ex2_approx(z0), p1 = ex2_approx(z1);
+    if constexpr (MASK) {
+      p0 = 2 * j < e_hi ? p0 : 0.f;
+      p1 = 2 * j + 1 < e_hi ? p1 : 0.f;
+    }
+    const uint64_t d2 = f2_mul(
+        f2_pack(p0, p1),
+        f2_add(f2_pack(__uint_as_float(dv[2 * j]), __uint_as_float(dv[2 * j + 1])), nd2));
+    float d0, d1;
+    f2_unpack(d2, d0, d1);
+    pd[jj] = bpack2<BF16>(d0, d1);
+  }
+  tmem_st8(t_d + hh * 8, pd);
+  }
 }
 
 // -------------------------------------------------------------------------------------------
@@ -223,6 +337,9 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     const int kl = threadIdx.x & 127;                   // key within the tile = TMEM lane
     const int key = key0 + kl;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    constexpr int BIAS = !ALIBI ? BIAS_NONE : (CAUSAL ? BIAS_LINEAR : BIAS_ABS);
+    const uint32_t stage = sb + C::SMEM_STAGE + static_cast<uint32_t>(warp) * 256u;
+    const uint64_t c1x2 = f2_pack(p.c1, p.c1);
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       ok = mbar_wait(TBAR(B_SF), it & 1, abort_flag, tmo, ecode | 5);
@@ -237,35 +354,49 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
 #pragma unroll 1
       for (int cc = 0; cc < C::CPW; ++cc) {
         const int c = C::CPW * wg + cc;       // 32-column chunk of the tile
-        uint32_t sv[32], dv[32];
-        tmem_ld32(t_lane + T_S + c * 32, sv);
-        tmem_ld32(t_lane + T_DP + c * 32, dv);
-        const int rr = row0 + c * 32 + lane;  // this lane fetches the row values of column rr
+        // The chunk's 32 S / dP columns in two halves of 16 (the second loaded once the first
+        // has been used), to stay within the registers of the 576-thread launch.
+        uint32_t sv[16], dv[16];
+        tmem_ld16(t_lane + T_S + c * 32, sv);
+        tmem_ld16(t_lane + T_DP + c * 32, dv);
+        // Lane e stages the terms of row rc0 + e for the whole warp (read back as broadcasts).
+        const int rc0 = row0 + c * 32;
+        const int rr = rc0 + lane;
         const size_t li = static_cast<size_t>(h) * p.total_q + q0 + rr;
-        const float lse_l = rr < lq ? __ldg(p.lse + li) * LOG2E : 0.f;
-        const float dl_l = rr < lq ? p.delta[li] : 0.f;
-        tmem_wait_ld();
-        uint32_t pp[16], pd[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pe[2], de[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int row = row0 + c * 32 + e + u;
-            const float lse_e = __shfl_sync(0xffffffffu, lse_l, e + u);
-            const float dl_e = __shfl_sync(0xffffffffu, dl_l, e + u);
-            const bool valid = row < lq && key < lk && (!CAUSAL || key <= row + shift);
-            float z = __uint_as_float(sv[e + u]) * p.c1 - lse_e;
-            if constexpr (ALIBI) z -= slope2 * fabsf(static_cast<float>(row + shift - key));
-            const float pv = valid ? ex2_approx(z) : 0.f;
-            pe[u] = pv;
-            de[u] = pv * (__uint_as_float(dv[e + u]) - dl_e);
-          }
-          pp[e >> 1] = bpack2<BF16>(pe[0], pe[1]);
-          pd[e >> 1] = bpack2<BF16>(de[0], de[1]);
+        float na = 0.f, nd = 0.f;
+        if (rr < lq) {
+          na = -__ldg(p.lse + li) * LOG2E;
+          if constexpr (BIAS == BIAS_LINEAR) na = fmaf(-slope2, static_cast<float>(lane), na);
+          nd = -p.delta[li];
         }
-        tmem_st16(t_lane + T_S + 32 * C::CPW * wg + cc * 16, pp);
-        tmem_st16(t_lane + T_DP + 32 * C::CPW * wg + cc * 16, pd);
+        __syncwarp();  // the previous chunk's reads of the staging area are done
+        sts_f32(stage + (lane >> 1) * 16u + (lane & 1) * 4u, na);
+        sts_f32(stage + (lane >> 1) * 16u + 8u + (lane & 1) * 4u, nd);
+        __syncwarp();
+        // rows rc0 + e with e_lo <= e < e_hi see this key
+        const int e_hi = key < lk ? min(32, lq - rc0) : 0;
+        const int e_lo = CAUSAL ? key - shift - rc0 : 0;
+        const bool full = __all_sync(0xffffffffu, e_lo <= 0 && e_hi >= 32);
+        const float dd = static_cast<float>(rc0 + shift - key);
+        const uint64_t kb2 = f2_pack(-slope2 * dd, -slope2 * dd);
+        tmem_wait_ld();
+        const uint32_t t_p = t_lane + T_S + 32 * C::CPW * wg + cc * 16;
+        const uint32_t t_d = t_lane + T_DP + 32 * C::CPW * wg + cc * 16;
+        if (full)
+          bwd_kv_half<BF16, false, BIAS, 0>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, t_p,
+                                            t_d);
+        else
+          bwd_kv_half<BF16, true, BIAS, 0>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, t_p,
+                                           t_d);
+        tmem_ld16(t_lane + T_S + c * 32 + 16, sv);
+        tmem_ld16(t_lane + T_DP + c * 32 + 16, dv);
+        tmem_wait_ld();
+        if (full)
+          bwd_kv_half<BF16, false, BIAS, 1>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, t_p,
+                                            t_d);
+        else
+          bwd_kv_half<BF16, true, BIAS, 1>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, t_p,
+                                           t_d);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -478,6 +609,9 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     const float dl = row < lq ? p.delta[li] : 0.f;
     float slope2 = 0.f;
     if constexpr (ALIBI) slope2 = __ldg(p.slopes + h) * LOG2E;
+    constexpr int BIAS = !ALIBI ? BIAS_NONE : (CAUSAL ? BIAS_LINEAR : BIAS_ABS);
+    const uint64_t c1x2 = f2_pack(p.c1, p.c1);
+    const uint64_t nd2 = f2_pack(-dl, -dl);
     bool ok = true;
     for (int jt = 0; jt < n_jt && ok; ++jt) {
       ok = mbar_wait(TBAR(B_SF), jt & 1, abort_flag, tmo, ecode | 5);
@@ -490,23 +624,22 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
         uint32_t sv[32], dv[32];
         tmem_ld32(t_lane + T_S + c * 32, sv);
         tmem_ld32(t_lane + T_DP + c * 32, dv);
+        // keys kc0 + e with e < e_hi are seen by this row
+        const int kc0 = jt * 128 + c * 32;
+        const int dk = row + shift - kc0;
+        int e_hi = row < lq ? min(32, lk - kc0) : 0;
+        if (CAUSAL) e_hi = min(e_hi, dk + 1);
+        const bool full = __all_sync(0xffffffffu, e_hi >= 32);
+        float b = -lse2;
+        if constexpr (BIAS == BIAS_LINEAR) b = fmaf(-slope2, static_cast<float>(dk), b);
         tmem_wait_ld();
-        uint32_t pd[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float de[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = jt * 128 + c * 32 + e + u;
-            const bool valid = row < lq && key < lk && (!CAUSAL || key <= row + shift);
-            float z = __uint_as_float(sv[e + u]) * p.c1 - lse2;
-            if constexpr (ALIBI) z -= slope2 * fabsf(static_cast<float>(row + shift - key));
-            const float pv = valid ? ex2_approx(z) : 0.f;
-            de[u] = pv * (__uint_as_float(dv[e + u]) - dl);
-          }
-          pd[e >> 1] = bpack2<BF16>(de[0], de[1]);
-        }
-        tmem_st16(t_lane + T_S + 32 * C::CPW * wg + cc * 16, pd);
+        const uint32_t t_d = t_lane + T_S + 32 * C::CPW * wg + cc * 16;
+        if (full)
+          bwd_q_chunk<BF16, false, BIAS>(sv, dv, c1x2, b, slope2, static_cast<float>(dk), nd2,
+                                         e_hi, t_d);
+        else
+          bwd_q_chunk<BF16, true, BIAS>(sv, dv, c1x2, b, slope2, static_cast<float>(dk), nd2,
+                                        e_hi, t_d);
       }
       tmem_wait_st();
       tc_fence_before();
