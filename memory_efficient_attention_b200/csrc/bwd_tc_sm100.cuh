@@ -18,7 +18,8 @@
 //
 // mea_bwd_dq_tc_kernel: one CTA per (128-row query tile, segment, query head), over the key
 // tiles the rows see: S = Q K^T, dP = dO V^T, dS (thread = row), dQ += dS K.
-// TMEM: S [0,128), dP [128,256), dQ [256,256+D).
+// TMEM: S(j) in [0,128) or [128,256) by the parity of j, dP [256,384), dQ [384,384+D); S(j+2)
+// is computed while the elementwise warps work on tile j+1.
 //
 // Roles (NWG*128 + 64 threads): NWG elementwise warpgroups (thread = TMEM lane; group w handles
 // the 32-column chunks [128w/NWG, 128(w+1)/NWG) of the S/dP tiles and writes its packed P / dS
@@ -454,6 +455,19 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
 }
 
 // -------------------------------------------------------------------------------------------
+// dQ kernel layout: Q and dO loaded once; K in a 3-stage ring (its last use, dQ(j), comes a tile
+// after S(j+2) would like to reuse the stage), V in a 2-stage ring (free after dP(j)).
+template <int D>
+struct BwdDqCfg {
+  using T = BwdTcCfg<D>;
+  static constexpr uint32_t SMEM_Q = 0, SMEM_DO = T::TILE_BYTES;
+  static constexpr uint32_t SMEM_K = 2 * T::TILE_BYTES;   // 3 stages
+  static constexpr uint32_t SMEM_V = 5 * T::TILE_BYTES;   // 2 stages
+  static constexpr uint32_t SMEM_BAR = 7 * T::TILE_BYTES;
+  static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
+  static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
+};
+
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
 __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     mea_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -462,6 +476,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
                          const __grid_constant__ CUtensorMap tm_v, const BwdParams p,
                          unsigned long long timeout_ns) {
   using C = BwdTcCfg<D>;
+  using L = BwdDqCfg<D>;
   constexpr float LOG2E = 1.4426950408889634f;
   // Causal: the last query tiles see the most keys; start them first.
   const int itile = CAUSAL ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
@@ -476,11 +491,14 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sb = smem_u32(smem);
-  constexpr int B_QD = 0, B_KF = 1, B_KE = 3, B_SF = 5, B_PF = 6, B_ACC = 7, B_DR = 8;
-  constexpr int N_BARS = 9;
-  const uint32_t bar0 = sb + C::SMEM_BAR;
+  // B_KF/B_KE: K ring (3), B_VF/B_VE: V ring (2); B_SF: S(j) and dP(j) in TMEM; B_PF: dS(j)
+  // packed by the elementwise warps (dP free again).
+  constexpr int B_QD = 0, B_KF = 1, B_KE = 4, B_VF = 7, B_VE = 9, B_SF = 11, B_PF = 12,
+                B_ACC = 13, B_DR = 14;
+  constexpr int N_BARS = 15;
+  const uint32_t bar0 = sb + L::SMEM_BAR;
 #define TBAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_BAR + 8 * N_BARS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SMEM_BAR + 8 * N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned ecode = (KID_BWD << 8) | 0x80;
@@ -496,9 +514,13 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(TBAR(B_QD), 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(TBAR(B_KF + b), 1);
       mbar_init(TBAR(B_KE + b), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(TBAR(B_VF + b), 1);
+      mbar_init(TBAR(B_VE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
     mbar_init(TBAR(B_PF), 4 * C::NWG);  // one elected arrival per elementwise warp
@@ -515,83 +537,102 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+  // TMEM: S(j) in buffer j mod 2, then dP and the dQ accumulator.
+  const uint32_t T_S0 = 0, T_DP = 256, T_DQ = 384;
 
   if (warp == C::W_LOAD) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t loaded = 0;
       bool ok = true;
+      int nk = 0, nv = 0;  // K / V loads issued
       mbar_arrive_expect_tx(TBAR(B_QD), 2 * C::TILE_BYTES);
 #pragma unroll
       for (int a = 0; a < C::ATOMS; ++a) {
-        tma_load_3d(sb + C::SMEM_A + a * C::ATOM_BYTES, &tm_q, TBAR(B_QD), a * 64, h, q0 + row0);
-        tma_load_3d(sb + C::SMEM_B + a * C::ATOM_BYTES, &tm_do, TBAR(B_QD), a * 64, h, q0 + row0);
+        tma_load_3d(sb + L::SMEM_Q + a * C::ATOM_BYTES, &tm_q, TBAR(B_QD), a * 64, h, q0 + row0);
+        tma_load_3d(sb + L::SMEM_DO + a * C::ATOM_BYTES, &tm_do, TBAR(B_QD), a * 64, h,
+                    q0 + row0);
       }
       for (int jt = 0; jt < n_jt && ok; ++jt) {
-        const int buf = jt & 1;
-        ok = mbar_wait(TBAR(B_KE + buf), ((jt >> 1) & 1) ^ 1, abort_flag, tmo, ecode | 1);
+        const int kb = jt % 3, vb = jt & 1;
+        ok = mbar_wait(TBAR(B_KE + kb), ((jt / 3) & 1) ^ 1, abort_flag, tmo, ecode | 1);
         if (!ok) break;
-        const uint32_t ks = sb + C::SMEM_RING + buf * 2 * C::TILE_BYTES;
-        mbar_arrive_expect_tx(TBAR(B_KF + buf), 2 * C::TILE_BYTES);
+        mbar_arrive_expect_tx(TBAR(B_KF + kb), C::TILE_BYTES);
 #pragma unroll
-        for (int a = 0; a < C::ATOMS; ++a) {
-          tma_load_3d(ks + a * C::ATOM_BYTES, &tm_k, TBAR(B_KF + buf), a * 64, g, k0 + jt * 128);
-          tma_load_3d(ks + C::TILE_BYTES + a * C::ATOM_BYTES, &tm_v, TBAR(B_KF + buf), a * 64, g,
-                      k0 + jt * 128);
-        }
-        ++loaded;
+        for (int a = 0; a < C::ATOMS; ++a)
+          tma_load_3d(sb + L::SMEM_K + kb * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_k,
+                      TBAR(B_KF + kb), a * 64, g, k0 + jt * 128);
+        nk = jt + 1;
+        ok = mbar_wait(TBAR(B_VE + vb), ((jt >> 1) & 1) ^ 1, abort_flag, tmo, ecode | 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(TBAR(B_VF + vb), C::TILE_BYTES);
+#pragma unroll
+        for (int a = 0; a < C::ATOMS; ++a)
+          tma_load_3d(sb + L::SMEM_V + vb * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_v,
+                      TBAR(B_VF + vb), a * 64, g, k0 + jt * 128);
+        nv = jt + 1;
       }
+      // Let every issued load land before shared memory goes away.
       volatile int never = 0;
       mbar_wait(TBAR(B_QD), 0, &never, tmo, ecode | 15);
-      for (uint32_t jt = (loaded > 2 ? loaded - 2 : 0); jt < loaded; ++jt)
-        mbar_wait(TBAR(B_KF + (jt & 1)), (jt >> 1) & 1, &never, tmo, ecode | 15);
+      for (int jt = max(0, nk - 3); jt < nk; ++jt)
+        mbar_wait(TBAR(B_KF + jt % 3), (jt / 3) & 1, &never, tmo, ecode | 15);
+      for (int jt = max(0, nv - 2); jt < nv; ++jt)
+        mbar_wait(TBAR(B_VF + (jt & 1)), (jt >> 1) & 1, &never, tmo, ecode | 15);
     }
   } else if (warp == C::W_ISSUE) {
     // ------------------------------------------------------------ tcgen05 issuer
+    // Order: S(0), dP(0), S(1); then per tile j, once dS(j) is packed: dP(j+1) (the next
+    // elementwise step can start after this one GEMM), dQ += dS(j) K(j), S(j+2) into the
+    // buffer dQ(j) has just read.
     if (lane == 0) {
       constexpr uint32_t ID_KK = umma_idesc_f16(BF16, 128, 128, false, false);
       constexpr uint32_t ID_PV = umma_idesc_f16(BF16, 128, D, false, true);
+      auto issue_s = [&](int jt) -> bool {
+        const int kb = jt % 3;
+        if (!mbar_wait(TBAR(B_KF + kb), (jt / 3) & 1, abort_flag, tmo, ecode | 3)) return false;
+        tc_fence_after();
+        const uint32_t ks = sb + L::SMEM_K + kb * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + T_S0 + (jt & 1) * 128, umma_desc_sw128(sb + L::SMEM_Q + off, 16, 1024),
+                 umma_desc_sw128(ks + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
+        }
+        return true;
+      };
+      auto issue_dp = [&](int jt) -> bool {
+        const int vb = jt & 1;
+        if (!mbar_wait(TBAR(B_VF + vb), (jt >> 1) & 1, abort_flag, tmo, ecode | 3)) return false;
+        tc_fence_after();
+        const uint32_t vs = sb + L::SMEM_V + vb * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + T_DP, umma_desc_sw128(sb + L::SMEM_DO + off, 16, 1024),
+                 umma_desc_sw128(vs + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(TBAR(B_VE + vb));
+        mma_commit(TBAR(B_SF));  // S(j) (issued earlier) and dP(j)
+        return true;
+      };
       bool ok = mbar_wait(TBAR(B_QD), 0, abort_flag, tmo, ecode | 2);
       tc_fence_after();
-      for (int jt = 0; jt <= n_jt && ok; ++jt) {
-        const int buf = jt & 1;
-        if (jt < n_jt) {
-          ok = mbar_wait(TBAR(B_KF + buf), (jt >> 1) & 1, abort_flag, tmo, ecode | 3);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        if (jt > 0) {
-          // ---- dQ += dS K for key tile jt-1
-          ok = mbar_wait_spin(TBAR(B_PF), (jt - 1) & 1, abort_flag, tmo, ecode | 4);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t ks = sb + C::SMEM_RING + ((jt - 1) & 1) * 2 * C::TILE_BYTES;
+      if (ok && n_jt > 0) ok = issue_s(0) && issue_dp(0);
+      if (ok && n_jt > 1) ok = issue_s(1);
+      for (int jt = 0; jt < n_jt && ok; ++jt) {
+        ok = mbar_wait_spin(TBAR(B_PF), jt & 1, abort_flag, tmo, ecode | 4);
+        if (!ok) break;
+        tc_fence_after();
+        if (jt + 1 < n_jt && !(ok = issue_dp(jt + 1))) break;
+        // ---- dQ += dS(j) K(j)
+        const uint32_t ks = sb + L::SMEM_K + (jt % 3) * C::TILE_BYTES;
 #pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16)
-            mma_ts(tmem + T_DQ, tmem + T_S + C::packed_col(k16),
-                   umma_desc_sw128(ks + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
-                   (jt - 1 > 0 || k16 > 0) ? 1u : 0u);
-          mma_commit(TBAR(B_KE + ((jt - 1) & 1)));
-        }
-        if (jt < n_jt) {
-          // ---- S = Q K^T, dP = dO V^T
-          const uint32_t ks = sb + C::SMEM_RING + buf * 2 * C::TILE_BYTES;
-          const uint32_t vs = ks + C::TILE_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-            mma_ss(tmem + T_S, umma_desc_sw128(sb + C::SMEM_A + off, 16, 1024),
-                   umma_desc_sw128(ks + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-            mma_ss(tmem + T_DP, umma_desc_sw128(sb + C::SMEM_B + off, 16, 1024),
-                   umma_desc_sw128(vs + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(TBAR(B_SF));
-        }
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_ts(tmem + T_DQ, tmem + T_S0 + (jt & 1) * 128 + C::packed_col(k16),
+                 umma_desc_sw128(ks + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
+                 (jt > 0 || k16 > 0) ? 1u : 0u);
+        mma_commit(TBAR(B_KE + jt % 3));
+        if (jt + 2 < n_jt && !(ok = issue_s(jt + 2))) break;
       }
       mma_commit(TBAR(B_ACC));
       mma_commit(TBAR(B_DR));
@@ -600,7 +641,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ elementwise (thread = row)
-    const int wg = threadIdx.x >> 7;                    // column half of this warpgroup
+    const int wg = threadIdx.x >> 7;                    // column quarter of this warpgroup
     const int rl = threadIdx.x & 127;
     const int row = row0 + rl;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -618,11 +659,12 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      const uint32_t t_s = T_S0 + (jt & 1) * 128;
 #pragma unroll 1
       for (int cc = 0; cc < C::CPW; ++cc) {
         const int c = C::CPW * wg + cc;
         uint32_t sv[32], dv[32];
-        tmem_ld32(t_lane + T_S + c * 32, sv);
+        tmem_ld32(t_lane + t_s + c * 32, sv);
         tmem_ld32(t_lane + T_DP + c * 32, dv);
         // keys kc0 + e with e < e_hi are seen by this row
         const int kc0 = jt * 128 + c * 32;
@@ -633,7 +675,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
         float b = -lse2;
         if constexpr (BIAS == BIAS_LINEAR) b = fmaf(-slope2, static_cast<float>(dk), b);
         tmem_wait_ld();
-        const uint32_t t_d = t_lane + T_S + 32 * C::CPW * wg + cc * 16;
+        const uint32_t t_d = t_lane + t_s + 32 * C::CPW * wg + cc * 16;
         if (full)
           bwd_q_chunk<BF16, false, BIAS>(sv, dv, c1x2, b, slope2, static_cast<float>(dk), nd2,
                                          e_hi, t_d);

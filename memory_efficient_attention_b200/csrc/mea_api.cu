@@ -310,9 +310,10 @@ template <int D, bool BF16, bool CAUSAL, bool ALIBI>
 int launch_bwd_t(const BwdMaps& m, const mea::BwdParams& p, int max_q, int max_k,
                  cudaStream_t stream) {
   constexpr uint32_t smem = mea::BwdTcCfg<D>::SMEM_TOTAL;
+  constexpr uint32_t smem_dq = mea::BwdDqCfg<D>::SMEM_TOTAL;
   constexpr auto kdkdv = mea::mea_bwd_dkdv_tc_kernel<D, BF16, CAUSAL, ALIBI>;
   constexpr auto kdq = mea::mea_bwd_dq_tc_kernel<D, BF16, CAUSAL, ALIBI>;
-  if (smem_attr_once<kdkdv>(smem) != cudaSuccess || smem_attr_once<kdq>(smem) != cudaSuccess)
+  if (smem_attr_once<kdkdv>(smem) != cudaSuccess || smem_attr_once<kdq>(smem_dq) != cudaSuccess)
     return MEA_ERR_CUDA;
   clear_stale_launch_error();
   const unsigned long long tmo = g_timeout_ns.load();
@@ -323,7 +324,7 @@ int launch_bwd_t(const BwdMaps& m, const mea::BwdParams& p, int max_q, int max_k
     kdkdv<<<dim3((max_k + 127) / 128, p.n_seqs, p.hkv), mea::BwdTcCfg<D>::THREADS, smem,
             stream>>>(m.q, m.dout, m.k, m.v, p, tmo);
   if (max_q > 0)
-    kdq<<<dim3((max_q + 127) / 128, p.n_seqs, p.hq), mea::BwdTcCfg<D>::THREADS, smem,
+    kdq<<<dim3((max_q + 127) / 128, p.n_seqs, p.hq), mea::BwdTcCfg<D>::THREADS, smem_dq,
           stream>>>(m.q, m.dout, m.k, m.v, p, tmo);
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
