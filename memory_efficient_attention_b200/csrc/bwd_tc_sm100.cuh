@@ -10,11 +10,14 @@
 // mea_bwd_dkdv_tc_kernel: one CTA per (128-key tile, segment, KV head). For every query tile of
 // the R heads of the group that sees the key tile:
 //   S^T = K Q^T, dP^T = V dO^T      (tcgen05, K-major operands, fp32 in TMEM)
-//   P^T, dS^T                        (elementwise warpgroup: thread = key = TMEM lane), written
-//                                    bf16/f16-packed over the first 64 columns of S^T / dP^T
-//   dV += P^T dO, dK += dS^T Q       (tcgen05, A from TMEM, B = the [rows][D] tiles MN-major)
+//   P^T, dS^T                        (elementwise warpgroup: thread = key = TMEM lane); dS^T
+//                                    16-bit-packed over the first 64 columns of dP^T, P^T into
+//                                    shared memory as a K-major operand
+//   dK += dS^T Q, dV += P^T dO       (tcgen05; A from TMEM / shared memory, B = the [rows][D]
+//                                    tiles MN-major)
 // TMEM: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D). dK and dV accumulate
-// over the whole GQA group; they are written once.
+// over the whole GQA group; they are written once. Since P^T does not sit in TMEM, S^T(i+1) is
+// computed while the elementwise warps still work on iteration i.
 //
 // mea_bwd_dq_tc_kernel: one CTA per (128-row query tile, segment, query head), over the key
 // tiles the rows see: S = Q K^T, dP = dO V^T, dS (thread = row), dQ += dS K.
@@ -24,8 +27,8 @@
 // Roles (NWG*128 + 64 threads): NWG elementwise warpgroups (thread = TMEM lane; group w handles
 // the 32-column chunks [128w/NWG, 128(w+1)/NWG) of the S/dP tiles and writes its packed P / dS
 // over the first half of its own columns, so the groups never touch each other's columns), warp
-// 4*NWG the tcgen05 issuer (owns TMEM), warp 4*NWG+1 the TMA producer. Every wait is bounded; no
-// named barriers in the role loops.
+// 4*NWG the tcgen05 issuer (owns TMEM), warp 4*NWG+1 the TMA producer. Every wait is bounded (all
+// hand-offs are mbarriers); no named barriers in the role loops.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -43,14 +46,6 @@ struct BwdTcCfg {
   static constexpr int ATOMS = D / 64;
   static constexpr uint32_t ATOM_BYTES = 128 * 128;      // 128 rows x 128 B
   static constexpr uint32_t TILE_BYTES = 128 * D * 2;
-  static constexpr uint32_t SMEM_A = 0;                  // K (dkdv) / Q (dq), loaded once
-  static constexpr uint32_t SMEM_B = TILE_BYTES;         // V (dkdv) / dO (dq), loaded once
-  static constexpr uint32_t SMEM_RING = 2 * TILE_BYTES;  // 2 stages x 2 tiles
-  static constexpr uint32_t SMEM_BAR = SMEM_RING + 4 * TILE_BYTES;
-  // 256 B per elementwise warp: the row terms of its current 32-row chunk (dK/dV kernel)
-  static constexpr uint32_t SMEM_STAGE = SMEM_BAR + 256;
-  static constexpr uint32_t SMEM_TOTAL = SMEM_STAGE + 4 * 4 * 256 + 1024;
-  static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
   static constexpr int NWG = 4;                          // elementwise warpgroups
   static constexpr int CPW = 4 / NWG;                      // 32-column chunks per group
   static constexpr int THREADS = NWG * 128 + 64;
@@ -88,19 +83,17 @@ enum { BIAS_NONE = 0, BIAS_LINEAR = 1, BIAS_ABS = 2 };
 // dK/dV elementwise step for half H (rows rc0 + 16H .. +15) of a 32-row chunk of the
 // S^T / dP^T tiles and this thread's key:
 //   p_e = 2^(c1 S_e + na_e + kb),  dS_e = p_e (dP_e + nd_e),  e = 0..31 (row rc0 + e)
-// with the row terms staged by the warp in shared memory as 16 float4 {na_e, na_e+1, nd_e,
-// nd_e+1}: na_e = -(lse_e log2 e) (BIAS_LINEAR: also - slope2 e), nd_e = -delta_e. kb is this
-// thread's key term (BIAS_LINEAR: -slope2 (rc0 + shift - key)); BIAS_ABS subtracts
-// slope2 |dabs + e| per element. MASK: p_e = 0 outside e_lo <= e < e_hi. sv / dv hold the
-// half's 16 S / dP columns. Pairs of columns go through the f32x2 pipe; P and dS leave packed
-// to 16 bits as eight words each, to TMEM at t_p + 8H and t_d + 8H (the chunk's own S / dP
-// columns, already read).
+// with the row terms staged in shared memory as 16 float4 {na_e, na_e+1, nd_e, nd_e+1}:
+// na_e = -(lse_e log2 e) (BIAS_LINEAR: also - slope2 e), nd_e = -delta_e. kb is this thread's
+// key term (BIAS_LINEAR: -slope2 (rc0 + shift - key)); BIAS_ABS subtracts slope2 |dabs + e| per
+// element. MASK: p_e = 0 outside e_lo <= e < e_hi. sv / dv hold the half's 16 S / dP columns.
+// Pairs of columns go through the f32x2 pipe; P and dS come out packed to 16 bits, eight words
+// each.
 template <bool BF16, bool MASK, int BIAS, int H>
 __device__ __forceinline__ void bwd_kv_half(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
                                             uint32_t stage, uint64_t c1x2, uint64_t kb2,
                                             float slope2, float dabs, int e_lo, int e_hi,
-                                            uint32_t t_p, uint32_t t_d) {
-  uint32_t pp[8], pd[8];
+                                            uint32_t (&pp)[8], uint32_t (&pd)[8]) {
 #pragma unroll
   for (int jj = 0; jj < 8; ++jj) {
     const int j = H * 8 + jj;  // column pair of the chunk
@@ -130,8 +123,6 @@ __device__ __forceinline__ void bwd_kv_half(const uint32_t (&sv)[16], const uint
     pp[jj] = bpack2<BF16>(p0, p1);
     pd[jj] = bpack2<BF16>(d0, d1);
   }
-  tmem_st8(t_p + H * 8, pp);
-  tmem_st8(t_d + H * 8, pd);
 }
 
 // dQ elementwise step for one 32-key chunk of the S / dP tiles and this thread's row:
@@ -183,6 +174,21 @@ __device__ __forceinline__ void bwd_q_chunk(const uint32_t (&sv)[32], const uint
 }
 
 // -------------------------------------------------------------------------------------------
+// dK/dV kernel layout: K and V loaded once; Q and dO in a 2-stage ring; P^T (128 keys x 128
+// query rows, 16-bit) written by the elementwise warps as the K-major, 128-byte-swizzled A
+// operand of dV += P^T dO; one 256-byte buffer per warpgroup for the row terms of its chunk.
+template <int D>
+struct BwdKvCfg {
+  using T = BwdTcCfg<D>;
+  static constexpr uint32_t SMEM_K = 0, SMEM_V = T::TILE_BYTES;
+  static constexpr uint32_t SMEM_RING = 2 * T::TILE_BYTES;  // 2 stages x (Q, dO)
+  static constexpr uint32_t SMEM_PT = 6 * T::TILE_BYTES;    // 2 atoms of 128 rows x 128 B
+  static constexpr uint32_t SMEM_BAR = SMEM_PT + 2 * T::ATOM_BYTES;
+  static constexpr uint32_t SMEM_STAGE = SMEM_BAR + 128;
+  static constexpr uint32_t SMEM_TOTAL = SMEM_STAGE + T::NWG * 256 + 1024;
+  static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
+};
+
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
 __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     mea_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -191,6 +197,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
                            const __grid_constant__ CUtensorMap tm_v, const BwdParams p,
                            unsigned long long timeout_ns) {
   using C = BwdTcCfg<D>;
+  using L = BwdKvCfg<D>;
+  static_assert(C::NWG == 4, "one 32-row chunk per elementwise warpgroup");
   constexpr float LOG2E = 1.4426950408889634f;
   const int jt = blockIdx.x, s = blockIdx.y, g = blockIdx.z;
   const int q0 = __ldg(p.cu_q + s), lq = __ldg(p.cu_q + s + 1) - q0;
@@ -202,11 +210,16 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sb = smem_u32(smem);
-  constexpr int B_KV = 0, B_QF = 1, B_QE = 3, B_SF = 5, B_PF = 6, B_ACC = 7, B_DR = 8;
-  constexpr int N_BARS = 9;
-  const uint32_t bar0 = sb + C::SMEM_BAR;
+  // B_SF: S^T(i), dP^T(i) in TMEM; B_SE: S^T(i) read by the elementwise warps (its columns may
+  // take S^T(i+1)); B_PF: P^T(i) in shared memory and dS^T(i) in TMEM; B_PTE: dV(i) has read
+  // P^T(i); B_STF: a warpgroup's row terms staged.
+  constexpr int B_KV = 0, B_QF = 1, B_QE = 3, B_SF = 5, B_SE = 6, B_PF = 7, B_PTE = 8,
+                B_ACC = 9, B_DR = 10, B_STF = 11;
+  constexpr int N_BARS = B_STF + C::NWG;
+  static_assert(8 * N_BARS + 8 <= 128, "barrier area");
+  const uint32_t bar0 = sb + L::SMEM_BAR;
 #define TBAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_BAR + 8 * N_BARS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SMEM_BAR + 8 * N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned ecode = KID_BWD << 8;
@@ -225,9 +238,12 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       mbar_init(TBAR(B_QE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
-    mbar_init(TBAR(B_PF), 4 * C::NWG);  // one elected arrival per elementwise warp
+    mbar_init(TBAR(B_SE), 4 * C::NWG);  // one elected arrival per elementwise warp
+    mbar_init(TBAR(B_PF), 4 * C::NWG);
+    mbar_init(TBAR(B_PTE), 1);
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
+    for (int w = 0; w < C::NWG; ++w) mbar_init(TBAR(B_STF + w), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -249,8 +265,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       mbar_arrive_expect_tx(TBAR(B_KV), 2 * C::TILE_BYTES);
 #pragma unroll
       for (int a = 0; a < C::ATOMS; ++a) {
-        tma_load_3d(sb + C::SMEM_A + a * C::ATOM_BYTES, &tm_k, TBAR(B_KV), a * 64, g, k0 + key0);
-        tma_load_3d(sb + C::SMEM_B + a * C::ATOM_BYTES, &tm_v, TBAR(B_KV), a * 64, g, k0 + key0);
+        tma_load_3d(sb + L::SMEM_K + a * C::ATOM_BYTES, &tm_k, TBAR(B_KV), a * 64, g, k0 + key0);
+        tma_load_3d(sb + L::SMEM_V + a * C::ATOM_BYTES, &tm_v, TBAR(B_KV), a * 64, g, k0 + key0);
       }
       for (int it = 0; it < n_iter && ok; ++it) {
         const int buf = it & 1;
@@ -259,7 +275,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
         const int r = it / nt, i = it0 + it % nt;
         const int h = g * p.R + r;
         const int row = q0 + i * 128;
-        const uint32_t qs = sb + C::SMEM_RING + buf * 2 * C::TILE_BYTES;
+        const uint32_t qs = sb + L::SMEM_RING + buf * 2 * C::TILE_BYTES;
         mbar_arrive_expect_tx(TBAR(B_QF + buf), 2 * C::TILE_BYTES);
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a) {
@@ -277,55 +293,74 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     }
   } else if (warp == C::W_ISSUE) {
     // ------------------------------------------------------------ tcgen05 issuer
+    // Order: S^T(0), dP^T(0); then per iteration i: S^T(i+1) once the elementwise warps have
+    // read S^T(i); once P^T(i) / dS^T(i) are out: dK(i), dP^T(i+1) (the next elementwise step
+    // waits for these two GEMMs only), then dV(i) from the shared-memory P^T.
     if (lane == 0) {
       constexpr uint32_t ID_KK = umma_idesc_f16(BF16, 128, 128, false, false);  // both K-major
       constexpr uint32_t ID_PV = umma_idesc_f16(BF16, 128, D, false, true);     // B MN-major
+      auto issue_st = [&](int it) {
+        const uint32_t qs = sb + L::SMEM_RING + (it & 1) * 2 * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + T_S, umma_desc_sw128(sb + L::SMEM_K + off, 16, 1024),
+                 umma_desc_sw128(qs + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_dpt = [&](int it) {
+        const uint32_t dos = sb + L::SMEM_RING + (it & 1) * 2 * C::TILE_BYTES + C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + T_DP, umma_desc_sw128(sb + L::SMEM_V + off, 16, 1024),
+                 umma_desc_sw128(dos + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(TBAR(B_SF));  // S^T(i) (issued earlier) and dP^T(i)
+      };
       bool ok = mbar_wait(TBAR(B_KV), 0, abort_flag, tmo, ecode | 2);
       tc_fence_after();
-      for (int it = 0; it <= n_iter && ok; ++it) {
-        const int buf = it & 1;
-        if (it < n_iter) {
-          ok = mbar_wait(TBAR(B_QF + buf), (it >> 1) & 1, abort_flag, tmo, ecode | 3);
+      if (ok && n_iter > 0) {
+        ok = mbar_wait(TBAR(B_QF), 0, abort_flag, tmo, ecode | 3);
+        tc_fence_after();
+        if (ok) {
+          issue_st(0);
+          issue_dpt(0);
+        }
+      }
+      for (int it = 0; it < n_iter && ok; ++it) {
+        if (it + 1 < n_iter) {
+          // ---- S^T(i+1) = K Q(i+1)^T into the columns S^T(i) was read from
+          ok = mbar_wait(TBAR(B_QF + ((it + 1) & 1)), ((it + 1) >> 1) & 1, abort_flag, tmo,
+                         ecode | 3);
+          if (ok) ok = mbar_wait_spin(TBAR(B_SE), it & 1, abort_flag, tmo, ecode | 7);
           if (!ok) break;
           tc_fence_after();
+          issue_st(it + 1);
         }
-        if (it > 0) {
-          // ---- dV += P^T dO, dK += dS^T Q for iteration it-1
-          ok = mbar_wait_spin(TBAR(B_PF), (it - 1) & 1, abort_flag, tmo, ecode | 4);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t qs = sb + C::SMEM_RING + ((it - 1) & 1) * 2 * C::TILE_BYTES;
-          const uint32_t dos = qs + C::TILE_BYTES;
+        ok = mbar_wait_spin(TBAR(B_PF), it & 1, abort_flag, tmo, ecode | 4);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t qs = sb + L::SMEM_RING + (it & 1) * 2 * C::TILE_BYTES;
+        const uint32_t dos = qs + C::TILE_BYTES;
+        // ---- dK += dS^T(i) Q(i)   (A: dS^T packed in TMEM)
 #pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16)
-            mma_ts(tmem + T_DV, tmem + T_S + C::packed_col(k16),
-                   umma_desc_sw128(dos + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
-                   (it - 1 > 0 || k16 > 0) ? 1u : 0u);
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_ts(tmem + T_DK, tmem + T_DP + C::packed_col(k16),
+                 umma_desc_sw128(qs + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
+                 (it > 0 || k16 > 0) ? 1u : 0u);
+        // ---- dP^T(i+1) = V dO(i+1)^T over the dS^T(i) columns dK has just read
+        if (it + 1 < n_iter) issue_dpt(it + 1);
+        // ---- dV += P^T(i) dO(i)   (A: P^T in shared memory, K-major)
 #pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16)
-            mma_ts(tmem + T_DK, tmem + T_DP + C::packed_col(k16),
-                   umma_desc_sw128(qs + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
-                   (it - 1 > 0 || k16 > 0) ? 1u : 0u);
-          mma_commit(TBAR(B_QE + ((it - 1) & 1)));
+        for (int k16 = 0; k16 < 8; ++k16) {
+          const uint32_t off = (k16 >> 2) * C::ATOM_BYTES + (k16 & 3) * 32;
+          mma_ss(tmem + T_DV, umma_desc_sw128(sb + L::SMEM_PT + off, 16, 1024),
+                 umma_desc_sw128(dos + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
+                 (it > 0 || k16 > 0) ? 1u : 0u);
         }
-        if (it < n_iter) {
-          // ---- S^T = K Q^T, dP^T = V dO^T
-          const uint32_t qs = sb + C::SMEM_RING + buf * 2 * C::TILE_BYTES;
-          const uint32_t dos = qs + C::TILE_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-            mma_ss(tmem + T_S, umma_desc_sw128(sb + C::SMEM_A + off, 16, 1024),
-                   umma_desc_sw128(qs + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-            mma_ss(tmem + T_DP, umma_desc_sw128(sb + C::SMEM_B + off, 16, 1024),
-                   umma_desc_sw128(dos + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(TBAR(B_SF));
-        }
+        mma_commit(TBAR(B_PTE));
+        mma_commit(TBAR(B_QE + (it & 1)));
       }
       mma_commit(TBAR(B_ACC));
       mma_commit(TBAR(B_DR));
@@ -334,13 +369,37 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ elementwise (thread = key)
-    const int wg = threadIdx.x >> 7;                    // column half of this warpgroup
+    const int wg = threadIdx.x >> 7;                    // 32-row chunk of this warpgroup
     const int kl = threadIdx.x & 127;                   // key within the tile = TMEM lane
     const int key = key0 + kl;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     constexpr int BIAS = !ALIBI ? BIAS_NONE : (CAUSAL ? BIAS_LINEAR : BIAS_ABS);
-    const uint32_t stage = sb + C::SMEM_STAGE + static_cast<uint32_t>(warp) * 256u;
+    const uint32_t stage = sb + L::SMEM_STAGE + static_cast<uint32_t>(wg) * 256u;
+    const bool stager = (warp & 3) == 0;  // stages the row terms for its warpgroup
+    // this thread's row of P^T: the chunk's 64 bytes in atom wg / 2, 16-byte units
+    // 4 (wg & 1) .. +3, 128-byte swizzle
+    const uint32_t pt_row = sb + L::SMEM_PT + static_cast<uint32_t>(wg >> 1) * C::ATOM_BYTES +
+                            static_cast<uint32_t>(kl) * 128u;
+    const uint32_t sw = static_cast<uint32_t>(kl & 7);
     const uint64_t c1x2 = f2_pack(p.c1, p.c1);
+    // Row terms of iteration i for this lane's row (loaded one iteration ahead by the stager).
+    auto row_terms = [&](int it, float& na, float& nd) {
+      na = 0.f;
+      nd = 0.f;
+      if (!stager || it >= n_iter) return;
+      const int r = it / nt, i = it0 + it % nt;
+      const int h = g * p.R + r;
+      const int rr = i * 128 + wg * 32 + lane;
+      if (rr < lq) {
+        const size_t li = static_cast<size_t>(h) * p.total_q + q0 + rr;
+        na = -__ldg(p.lse + li) * LOG2E;
+        if constexpr (BIAS == BIAS_LINEAR)
+          na = fmaf(-__ldg(p.slopes + h) * LOG2E, static_cast<float>(lane), na);
+        nd = -p.delta[li];
+      }
+    };
+    float na_n, nd_n;
+    row_terms(0, na_n, nd_n);
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       ok = mbar_wait(TBAR(B_SF), it & 1, abort_flag, tmo, ecode | 5);
@@ -352,54 +411,62 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       const int row0 = i * 128;
       float slope2 = 0.f;
       if constexpr (ALIBI) slope2 = __ldg(p.slopes + h) * LOG2E;
-#pragma unroll 1
-      for (int cc = 0; cc < C::CPW; ++cc) {
-        const int c = C::CPW * wg + cc;       // 32-column chunk of the tile
-        // The chunk's 32 S / dP columns in two halves of 16 (the second loaded once the first
-        // has been used), to stay within the registers of the 576-thread launch.
-        uint32_t sv[16], dv[16];
-        tmem_ld16(t_lane + T_S + c * 32, sv);
-        tmem_ld16(t_lane + T_DP + c * 32, dv);
-        // Lane e stages the terms of row rc0 + e for the whole warp (read back as broadcasts).
-        const int rc0 = row0 + c * 32;
-        const int rr = rc0 + lane;
-        const size_t li = static_cast<size_t>(h) * p.total_q + q0 + rr;
-        float na = 0.f, nd = 0.f;
-        if (rr < lq) {
-          na = -__ldg(p.lse + li) * LOG2E;
-          if constexpr (BIAS == BIAS_LINEAR) na = fmaf(-slope2, static_cast<float>(lane), na);
-          nd = -p.delta[li];
-        }
-        __syncwarp();  // the previous chunk's reads of the staging area are done
-        sts_f32(stage + (lane >> 1) * 16u + (lane & 1) * 4u, na);
-        sts_f32(stage + (lane >> 1) * 16u + 8u + (lane & 1) * 4u, nd);
+      const int rc0 = row0 + wg * 32;  // first row of this warpgroup's chunk
+      uint32_t sv[16], dv[16];
+      tmem_ld16(t_lane + T_S + wg * 32, sv);
+      tmem_ld16(t_lane + T_DP + wg * 32, dv);
+      // Every warp finished reading the previous staged terms before B_SF (it waits for all
+      // elementwise warps' B_PF), so the stager may overwrite them now.
+      if (stager) {
+        sts_f32(stage + (lane >> 1) * 16u + (lane & 1) * 4u, na_n);
+        sts_f32(stage + (lane >> 1) * 16u + 8u + (lane & 1) * 4u, nd_n);
         __syncwarp();
-        // rows rc0 + e with e_lo <= e < e_hi see this key
-        const int e_hi = key < lk ? min(32, lq - rc0) : 0;
-        const int e_lo = CAUSAL ? key - shift - rc0 : 0;
-        const bool full = __all_sync(0xffffffffu, e_lo <= 0 && e_hi >= 32);
-        const float dd = static_cast<float>(rc0 + shift - key);
-        const uint64_t kb2 = f2_pack(-slope2 * dd, -slope2 * dd);
-        tmem_wait_ld();
-        const uint32_t t_p = t_lane + T_S + 32 * C::CPW * wg + cc * 16;
-        const uint32_t t_d = t_lane + T_DP + 32 * C::CPW * wg + cc * 16;
-        if (full)
-          bwd_kv_half<BF16, false, BIAS, 0>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, t_p,
-                                            t_d);
-        else
-          bwd_kv_half<BF16, true, BIAS, 0>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, t_p,
-                                           t_d);
-        tmem_ld16(t_lane + T_S + c * 32 + 16, sv);
-        tmem_ld16(t_lane + T_DP + c * 32 + 16, dv);
-        tmem_wait_ld();
-        if (full)
-          bwd_kv_half<BF16, false, BIAS, 1>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, t_p,
-                                            t_d);
-        else
-          bwd_kv_half<BF16, true, BIAS, 1>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, t_p,
-                                           t_d);
+        if (lane == 0) mbar_arrive(TBAR(B_STF + wg));
+        row_terms(it + 1, na_n, nd_n);
       }
+      // rows rc0 + e with e_lo <= e < e_hi see this key
+      const int e_hi = key < lk ? min(32, lq - rc0) : 0;
+      const int e_lo = CAUSAL ? key - shift - rc0 : 0;
+      const bool full = __all_sync(0xffffffffu, e_lo <= 0 && e_hi >= 32);
+      const float dd = static_cast<float>(rc0 + shift - key);
+      const uint64_t kb2 = f2_pack(-slope2 * dd, -slope2 * dd);
+      ok = mbar_wait(TBAR(B_STF + wg), it & 1, abort_flag, tmo, ecode | 8);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tmem_wait_ld();
+      uint32_t pp[8], pd[8];
+      if (full)
+        bwd_kv_half<BF16, false, BIAS, 0>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, pp, pd);
+      else
+        bwd_kv_half<BF16, true, BIAS, 0>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, pp, pd);
+      tmem_st8(t_lane + T_DP + wg * 32, pd);
+      // The second half of the chunk's S^T / dP^T columns; once it has landed S^T(i) is free.
+      tmem_ld16(t_lane + T_S + wg * 32 + 16, sv);
+      tmem_ld16(t_lane + T_DP + wg * 32 + 16, dv);
+      // P^T(i-1) has been read by dV(i-1) before P^T(i) goes over it.
+      ok = mbar_wait(TBAR(B_PTE), (it - 1) & 1, abort_flag, tmo, ecode | 9);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + 0) ^ sw) << 4), pp[0], pp[1],
+                   pp[2], pp[3]);
+      st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + 1) ^ sw) << 4), pp[4], pp[5],
+                   pp[6], pp[7]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(TBAR(B_SE));
+      if (full)
+        bwd_kv_half<BF16, false, BIAS, 1>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, pp, pd);
+      else
+        bwd_kv_half<BF16, true, BIAS, 1>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, pp, pd);
+      tmem_st8(t_lane + T_DP + wg * 32 + 8, pd);
+      st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + 2) ^ sw) << 4), pp[0], pp[1],
+                   pp[2], pp[3]);
+      st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + 3) ^ sw) << 4), pp[4], pp[5],
+                   pp[6], pp[7]);
+      // dS^T in TMEM and P^T in shared memory (generic proxy) reach the tensor core's reads.
       tmem_wait_st();
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(TBAR(B_PF));

@@ -309,7 +309,7 @@ struct BwdMaps {
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
 int launch_bwd_t(const BwdMaps& m, const mea::BwdParams& p, int max_q, int max_k,
                  cudaStream_t stream) {
-  constexpr uint32_t smem = mea::BwdTcCfg<D>::SMEM_TOTAL;
+  constexpr uint32_t smem = mea::BwdKvCfg<D>::SMEM_TOTAL;
   constexpr uint32_t smem_dq = mea::BwdDqCfg<D>::SMEM_TOTAL;
   constexpr auto kdkdv = mea::mea_bwd_dkdv_tc_kernel<D, BF16, CAUSAL, ALIBI>;
   constexpr auto kdq = mea::mea_bwd_dq_tc_kernel<D, BF16, CAUSAL, ALIBI>;
