@@ -186,8 +186,9 @@ int mea_forward_fp8(const void* q, const void* k, const void* v, void* out, floa
                     void* stream);
 
 /*
- * mea_backward_workspace_size — bytes of workspace mea_backward needs: one fp32 per (query head,
- * query token) for delta = rowsum(dout * out), plus 256 bytes of alignment slack.
+ * mea_backward_workspace_size — bytes of workspace mea_backward needs: two fp32 per (query
+ * head, query token) and per each of 128 pad rows a head (delta = rowsum(dout * out) and the
+ * row's exponent term, computed by the first kernel), plus 256 bytes of alignment slack.
  */
 size_t mea_backward_workspace_size(int total_q, int n_heads_q);
 

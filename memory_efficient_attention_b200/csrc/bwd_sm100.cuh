@@ -2,8 +2,12 @@
 //
 // The backward computes dq, dk, dv of L = sum(out * dout) for the forward's definition; its
 // main kernels (tcgen05) are in bwd_tc_sm100.cuh. This file holds the parameter block and
-//   mea_bwd_pre_kernel   delta[h, t] = rowsum(dO * O) in fp32, one warp per (token, head) row
-//                        (HBM-bound: reads out and dout once).
+//   mea_bwd_pre_kernel   per (query head, token) row, one warp each (HBM-bound: reads out and
+//                        dout once): nd = -rowsum(dO * O) = -delta and the row's exponent term
+//                        na = -lse log2 e (causal ALiBi: also - slope log2 e ((t - q0) mod 32),
+//                        t - q0 the row's index in its segment), both fp32 in the workspace.
+//                        128 zero rows per head follow the last token, so the tile loops of
+//                        the dK/dV kernel may read row terms up to a tile past a segment's end.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -23,7 +27,10 @@ struct BwdParams {
   void* dq;
   void* dk;
   void* dv;
-  float* delta;         // [Hq, T_q] workspace
+  float* nd;            // [Hq, t_pad] workspace: -delta of each row (zero in the pad rows)
+  float* na;            // [Hq, t_pad] workspace: the row's exponent term (see the pre kernel)
+  int t_pad;            // total_q + 128
+  int lin_bias;         // causal ALiBi: na carries -slope log2 e ((t - q0) mod 32)
   const int32_t* cu_q;
   const int32_t* cu_k;
   const float* slopes;  // [Hq] natural-log ALiBi slopes, or null
@@ -43,8 +50,16 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(128) mea_bwd_pre_kernel(const BwdParams p) {
   const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= static_cast<long long>(p.total_q) * p.hq) return;
+  if (row >= static_cast<long long>(p.t_pad) * p.hq) return;
   const int t = static_cast<int>(row / p.hq), h = static_cast<int>(row % p.hq);
+  const size_t wi = static_cast<size_t>(h) * p.t_pad + t;
+  if (t >= p.total_q) {  // pad row
+    if (lane == 0) {
+      p.nd[wi] = 0.f;
+      p.na[wi] = 0.f;
+    }
+    return;
+  }
   // lane takes the element pairs 2*lane + 64*i of the row's dh (even) elements
   const size_t base = (static_cast<size_t>(t) * p.hq + h) * p.dh;
   const uint16_t* o = reinterpret_cast<const uint16_t*>(p.out) + base;
@@ -71,7 +86,22 @@ __global__ void __launch_bounds__(128) mea_bwd_pre_kernel(const BwdParams p) {
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) p.delta[static_cast<size_t>(h) * p.total_q + t] = acc;
+  if (lane == 0) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    float na = -__ldg(p.lse + static_cast<size_t>(h) * p.total_q + t) * LOG2E;
+    if (p.lin_bias) {
+      // start of the token's segment: the last s with cu_q[s] <= t
+      int lo = 0, hi = p.n_seqs;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(p.cu_q + mid) <= t) lo = mid; else hi = mid;
+      }
+      const int e = (t - __ldg(p.cu_q + lo)) & 31;
+      na = fmaf(-__ldg(p.slopes + h) * LOG2E, static_cast<float>(e), na);
+    }
+    p.nd[wi] = -acc;
+    p.na[wi] = na;
+  }
 }
 
 }  // namespace mea

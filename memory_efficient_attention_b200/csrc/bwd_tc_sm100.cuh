@@ -65,44 +65,28 @@ __device__ __forceinline__ uint32_t bpack2(float lo, float hi) {
   return dpack2<BF16>(lo, hi);
 }
 
-__device__ __forceinline__ void lds_f4(uint32_t addr, float& a, float& b, float& c, float& d) {
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(a), "=f"(b), "=f"(c), "=f"(d)
-               : "r"(addr)
-               : "memory");
-}
-__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
-  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
 // Bias forms of the scores: none, causal ALiBi (the distance row + shift - key is >= 0 wherever
 // p can be non-zero, so the bias is linear in row and key), ALiBi without the causal mask
 // (|row + shift - key|).
 enum { BIAS_NONE = 0, BIAS_LINEAR = 1, BIAS_ABS = 2 };
 
-// dK/dV elementwise step for half H (rows rc0 + 16H .. +15) of a 32-row chunk of the
-// S^T / dP^T tiles and this thread's key:
-//   p_e = 2^(c1 S_e + na_e + kb),  dS_e = p_e (dP_e + nd_e),  e = 0..31 (row rc0 + e)
-// with the row terms staged in shared memory as 16 float4 {na_e, na_e+1, nd_e, nd_e+1}:
-// na_e = -(lse_e log2 e) (BIAS_LINEAR: also - slope2 e), nd_e = -delta_e. kb is this thread's
-// key term (BIAS_LINEAR: -slope2 (rc0 + shift - key)); BIAS_ABS subtracts slope2 |dabs + e| per
-// element. MASK: p_e = 0 outside e_lo <= e < e_hi. sv / dv hold the half's 16 S / dP columns.
-// Pairs of columns go through the f32x2 pipe; P and dS come out packed to 16 bits, eight words
-// each.
-template <bool BF16, bool MASK, int BIAS, int H>
-__device__ __forceinline__ void bwd_kv_half(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
-                                            uint32_t stage, uint64_t c1x2, uint64_t kb2,
-                                            float slope2, float dabs, int e_lo, int e_hi,
-                                            uint32_t (&pp)[8], uint32_t (&pd)[8]) {
+// dK/dV elementwise step, phase A, for a 32-row chunk of S^T and this thread's key:
+//   p_e = 2^(c1 S_e + na_e + kb),  e = 0..31 (row rc0 + e)
+// with na_e the row's exponent term from the pre kernel (-lse log2 e; causal ALiBi also
+// - slope2 e) read at na_row[e] (the same address in every lane: one broadcast load), kb this
+// thread's key term (BIAS_LINEAR: -slope2 (rc0 + shift - key)); BIAS_ABS subtracts
+// slope2 |dabs + e| per element. MASK: p_e = 0 outside e_lo <= e < e_hi. Pairs of columns go
+// through the f32x2 pipe.
+template <bool MASK, int BIAS>
+__device__ __forceinline__ void bwd_kv_p(const uint32_t (&sv)[32], const float* na_row,
+                                         uint64_t c1x2, uint64_t kb2, float slope2, float dabs,
+                                         int e_lo, int e_hi, float (&pr)[32]) {
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
-    const int j = H * 8 + jj;  // column pair of the chunk
-    float na0, na1, nd0, nd1;
-    lds_f4(stage + 16u * j, na0, na1, nd0, nd1);
-    uint64_t b2 = f2_pack(na0, na1);
+  for (int j = 0; j < 16; ++j) {
+    uint64_t b2 = f2_pack(__ldg(na_row + 2 * j), __ldg(na_row + 2 * j + 1));
     if constexpr (BIAS == BIAS_LINEAR) b2 = f2_add(b2, kb2);
     const uint64_t z2 =
-        f2_fma(f2_pack(__uint_as_float(sv[2 * jj]), __uint_as_float(sv[2 * jj + 1])), c1x2, b2);
+        f2_fma(f2_pack(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), c1x2, b2);
     float z0, z1;
     f2_unpack(z2, z0, z1);
     if constexpr (BIAS == BIAS_ABS) {
@@ -114,13 +98,26 @@ __device__ __forceinline__ void bwd_kv_half(const uint32_t (&sv)[16], const uint
       p0 = (2 * j >= e_lo && 2 * j < e_hi) ? p0 : 0.f;
       p1 = (2 * j + 1 >= e_lo && 2 * j + 1 < e_hi) ? p1 : 0.f;
     }
+    pr[2 * j] = p0;
+    pr[2 * j + 1] = p1;
+  }
+}
+
+// Phase B for half H (rows 16H .. 16H+15 of the chunk): dS_e = p_e (dP_e + nd_e) with
+// nd_e = -delta_e from the pre kernel (broadcast loads at nd_row[e]); dv holds the half's 16
+// dP^T columns; dS comes out packed to 16 bits, eight words.
+template <bool BF16, int H>
+__device__ __forceinline__ void bwd_kv_ds(const float (&pr)[32], const uint32_t (&dv)[16],
+                                          const float* nd_row, uint32_t (&pd)[8]) {
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int j = H * 8 + jj;
     const uint64_t d2 = f2_mul(
-        f2_pack(p0, p1),
+        f2_pack(pr[2 * j], pr[2 * j + 1]),
         f2_add(f2_pack(__uint_as_float(dv[2 * jj]), __uint_as_float(dv[2 * jj + 1])),
-               f2_pack(nd0, nd1)));
+               f2_pack(__ldg(nd_row + 2 * j), __ldg(nd_row + 2 * j + 1))));
     float d0, d1;
     f2_unpack(d2, d0, d1);
-    pp[jj] = bpack2<BF16>(p0, p1);
     pd[jj] = bpack2<BF16>(d0, d1);
   }
 }
@@ -176,7 +173,7 @@ __device__ __forceinline__ void bwd_q_chunk(const uint32_t (&sv)[32], const uint
 // -------------------------------------------------------------------------------------------
 // dK/dV kernel layout: K and V loaded once; Q and dO in a 2-stage ring; P^T (128 keys x 128
 // query rows, 16-bit) written by the elementwise warps as the K-major, 128-byte-swizzled A
-// operand of dV += P^T dO; one 256-byte buffer per warpgroup for the row terms of its chunk.
+// operand of dV += P^T dO.
 template <int D>
 struct BwdKvCfg {
   using T = BwdTcCfg<D>;
@@ -184,8 +181,7 @@ struct BwdKvCfg {
   static constexpr uint32_t SMEM_RING = 2 * T::TILE_BYTES;  // 2 stages x (Q, dO)
   static constexpr uint32_t SMEM_PT = 6 * T::TILE_BYTES;    // 2 atoms of 128 rows x 128 B
   static constexpr uint32_t SMEM_BAR = SMEM_PT + 2 * T::ATOM_BYTES;
-  static constexpr uint32_t SMEM_STAGE = SMEM_BAR + 128;
-  static constexpr uint32_t SMEM_TOTAL = SMEM_STAGE + T::NWG * 256 + 1024;
+  static constexpr uint32_t SMEM_TOTAL = SMEM_BAR + 256 + 1024;
   static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
 };
 
@@ -210,13 +206,15 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sb = smem_u32(smem);
-  // B_SF: S^T(i), dP^T(i) in TMEM; B_SE: S^T(i) read by the elementwise warps (its columns may
-  // take S^T(i+1)); B_PF: P^T(i) in shared memory and dS^T(i) in TMEM; B_PTE: dV(i) has read
-  // P^T(i); B_STF: a warpgroup's row terms staged.
-  constexpr int B_KV = 0, B_QF = 1, B_QE = 3, B_SF = 5, B_SE = 6, B_PF = 7, B_PTE = 8,
-                B_ACC = 9, B_DR = 10, B_STF = 11;
-  constexpr int N_BARS = B_STF + C::NWG;
-  static_assert(8 * N_BARS + 8 <= 128, "barrier area");
+  // B_QF/B_QE, B_DF/B_DE: the Q and dO halves of the 2-stage ring, full / empty (Q is free once
+  // dK(i) has read it, which is well before dV(i) frees dO, so Q(i+2) starts loading early);
+  // B_STR: S^T(i) in TMEM; B_SF: dP^T(i) in TMEM (and dK(i-1) done); B_SE: S^T(i) read by the
+  // elementwise warps (its columns may take S^T(i+1)); B_PF: P^T(i) in shared memory and dS^T(i)
+  // in TMEM; B_PTE: dV(i) has read P^T(i).
+  constexpr int B_KV = 0, B_QF = 1, B_QE = 3, B_DF = 5, B_DE = 7, B_SF = 9, B_SE = 10,
+                B_PF = 11, B_PTE = 12, B_ACC = 13, B_DR = 14, B_STR = 15;
+  constexpr int N_BARS = 16;
+  static_assert(8 * N_BARS + 8 <= 256, "barrier area");
   const uint32_t bar0 = sb + L::SMEM_BAR;
 #define TBAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SMEM_BAR + 8 * N_BARS);
@@ -236,6 +234,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(TBAR(B_QF + b), 1);
       mbar_init(TBAR(B_QE + b), 1);
+      mbar_init(TBAR(B_DF + b), 1);
+      mbar_init(TBAR(B_DE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
     mbar_init(TBAR(B_SE), 4 * C::NWG);  // one elected arrival per elementwise warp
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     mbar_init(TBAR(B_PTE), 1);
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
-    for (int w = 0; w < C::NWG; ++w) mbar_init(TBAR(B_STF + w), 1);
+    mbar_init(TBAR(B_STR), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -259,43 +259,50 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
 
   if (warp == C::W_LOAD) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // lane 0: K, V, then the Q tiles; lane 1: the dO tiles (each on its own ring barriers)
+    if (lane < 2) {
+      const bool is_q = lane == 0;
+      const int FB = is_q ? B_QF : B_DF, EB = is_q ? B_QE : B_DE;
+      const CUtensorMap* tm = is_q ? &tm_q : &tm_do;
+      const uint32_t off = is_q ? 0u : C::TILE_BYTES;
       uint32_t loaded = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(TBAR(B_KV), 2 * C::TILE_BYTES);
+      if (is_q) {
+        mbar_arrive_expect_tx(TBAR(B_KV), 2 * C::TILE_BYTES);
 #pragma unroll
-      for (int a = 0; a < C::ATOMS; ++a) {
-        tma_load_3d(sb + L::SMEM_K + a * C::ATOM_BYTES, &tm_k, TBAR(B_KV), a * 64, g, k0 + key0);
-        tma_load_3d(sb + L::SMEM_V + a * C::ATOM_BYTES, &tm_v, TBAR(B_KV), a * 64, g, k0 + key0);
+        for (int a = 0; a < C::ATOMS; ++a) {
+          tma_load_3d(sb + L::SMEM_K + a * C::ATOM_BYTES, &tm_k, TBAR(B_KV), a * 64, g,
+                      k0 + key0);
+          tma_load_3d(sb + L::SMEM_V + a * C::ATOM_BYTES, &tm_v, TBAR(B_KV), a * 64, g,
+                      k0 + key0);
+        }
       }
       for (int it = 0; it < n_iter && ok; ++it) {
         const int buf = it & 1;
-        ok = mbar_wait(TBAR(B_QE + buf), ((it >> 1) & 1) ^ 1, abort_flag, tmo, ecode | 1);
+        ok = mbar_wait(TBAR(EB + buf), ((it >> 1) & 1) ^ 1, abort_flag, tmo, ecode | 1);
         if (!ok) break;
         const int r = it / nt, i = it0 + it % nt;
         const int h = g * p.R + r;
         const int row = q0 + i * 128;
-        const uint32_t qs = sb + L::SMEM_RING + buf * 2 * C::TILE_BYTES;
-        mbar_arrive_expect_tx(TBAR(B_QF + buf), 2 * C::TILE_BYTES);
+        const uint32_t dst = sb + L::SMEM_RING + buf * 2 * C::TILE_BYTES + off;
+        mbar_arrive_expect_tx(TBAR(FB + buf), C::TILE_BYTES);
 #pragma unroll
-        for (int a = 0; a < C::ATOMS; ++a) {
-          tma_load_3d(qs + a * C::ATOM_BYTES, &tm_q, TBAR(B_QF + buf), a * 64, h, row);
-          tma_load_3d(qs + C::TILE_BYTES + a * C::ATOM_BYTES, &tm_do, TBAR(B_QF + buf), a * 64, h,
-                      row);
-        }
+        for (int a = 0; a < C::ATOMS; ++a)
+          tma_load_3d(dst + a * C::ATOM_BYTES, tm, TBAR(FB + buf), a * 64, h, row);
         ++loaded;
       }
       // Let every issued load land before shared memory goes away.
       volatile int never = 0;
-      mbar_wait(TBAR(B_KV), 0, &never, tmo, ecode | 15);
+      if (is_q) mbar_wait(TBAR(B_KV), 0, &never, tmo, ecode | 15);
       for (uint32_t it = (loaded > 2 ? loaded - 2 : 0); it < loaded; ++it)
-        mbar_wait(TBAR(B_QF + (it & 1)), (it >> 1) & 1, &never, tmo, ecode | 15);
+        mbar_wait(TBAR(FB + (it & 1)), (it >> 1) & 1, &never, tmo, ecode | 15);
     }
   } else if (warp == C::W_ISSUE) {
     // ------------------------------------------------------------ tcgen05 issuer
     // Order: S^T(0), dP^T(0); then per iteration i: S^T(i+1) once the elementwise warps have
-    // read S^T(i); once P^T(i) / dS^T(i) are out: dK(i), dP^T(i+1) (the next elementwise step
-    // waits for these two GEMMs only), then dV(i) from the shared-memory P^T.
+    // read S^T(i) (they exponentiate it while the tensor core runs the rest); once P^T(i) /
+    // dS^T(i) are out: dK(i), dP^T(i+1) (the second phase of the next elementwise step waits
+    // for these two GEMMs only), then dV(i) from the shared-memory P^T.
     if (lane == 0) {
       constexpr uint32_t ID_KK = umma_idesc_f16(BF16, 128, 128, false, false);  // both K-major
       constexpr uint32_t ID_PV = umma_idesc_f16(BF16, 128, D, false, true);     // B MN-major
@@ -307,6 +314,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
           mma_ss(tmem + T_S, umma_desc_sw128(sb + L::SMEM_K + off, 16, 1024),
                  umma_desc_sw128(qs + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
         }
+        mma_commit(TBAR(B_STR));
       };
       auto issue_dpt = [&](int it) {
         const uint32_t dos = sb + L::SMEM_RING + (it & 1) * 2 * C::TILE_BYTES + C::TILE_BYTES;
@@ -316,17 +324,17 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
           mma_ss(tmem + T_DP, umma_desc_sw128(sb + L::SMEM_V + off, 16, 1024),
                  umma_desc_sw128(dos + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(TBAR(B_SF));  // S^T(i) (issued earlier) and dP^T(i)
+        mma_commit(TBAR(B_SF));  // dP^T(i) (and everything issued before it)
       };
       bool ok = mbar_wait(TBAR(B_KV), 0, abort_flag, tmo, ecode | 2);
       tc_fence_after();
       if (ok && n_iter > 0) {
         ok = mbar_wait(TBAR(B_QF), 0, abort_flag, tmo, ecode | 3);
         tc_fence_after();
-        if (ok) {
-          issue_st(0);
-          issue_dpt(0);
-        }
+        if (ok) issue_st(0);
+        if (ok) ok = mbar_wait(TBAR(B_DF), 0, abort_flag, tmo, ecode | 3);
+        tc_fence_after();
+        if (ok) issue_dpt(0);
       }
       for (int it = 0; it < n_iter && ok; ++it) {
         if (it + 1 < n_iter) {
@@ -343,14 +351,21 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
         tc_fence_after();
         const uint32_t qs = sb + L::SMEM_RING + (it & 1) * 2 * C::TILE_BYTES;
         const uint32_t dos = qs + C::TILE_BYTES;
-        // ---- dK += dS^T(i) Q(i)   (A: dS^T packed in TMEM)
+        // ---- dK += dS^T(i) Q(i)   (A: dS^T packed in TMEM); the last read of Q(i)
 #pragma unroll
         for (int k16 = 0; k16 < 8; ++k16)
           mma_ts(tmem + T_DK, tmem + T_DP + C::packed_col(k16),
                  umma_desc_sw128(qs + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
                  (it > 0 || k16 > 0) ? 1u : 0u);
+        mma_commit(TBAR(B_QE + (it & 1)));
         // ---- dP^T(i+1) = V dO(i+1)^T over the dS^T(i) columns dK has just read
-        if (it + 1 < n_iter) issue_dpt(it + 1);
+        if (it + 1 < n_iter) {
+          ok = mbar_wait(TBAR(B_DF + ((it + 1) & 1)), ((it + 1) >> 1) & 1, abort_flag, tmo,
+                         ecode | 3);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dpt(it + 1);
+        }
         // ---- dV += P^T(i) dO(i)   (A: P^T in shared memory, K-major)
 #pragma unroll
         for (int k16 = 0; k16 < 8; ++k16) {
@@ -360,7 +375,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
                  (it > 0 || k16 > 0) ? 1u : 0u);
         }
         mma_commit(TBAR(B_PTE));
-        mma_commit(TBAR(B_QE + (it & 1)));
+        mma_commit(TBAR(B_DE + (it & 1)));
       }
       mma_commit(TBAR(B_ACC));
       mma_commit(TBAR(B_DR));
@@ -374,96 +389,84 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     const int key = key0 + kl;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     constexpr int BIAS = !ALIBI ? BIAS_NONE : (CAUSAL ? BIAS_LINEAR : BIAS_ABS);
-    const uint32_t stage = sb + L::SMEM_STAGE + static_cast<uint32_t>(wg) * 256u;
-    const bool stager = (warp & 3) == 0;  // stages the row terms for its warpgroup
     // this thread's row of P^T: the chunk's 64 bytes in atom wg / 2, 16-byte units
     // 4 (wg & 1) .. +3, 128-byte swizzle
     const uint32_t pt_row = sb + L::SMEM_PT + static_cast<uint32_t>(wg >> 1) * C::ATOM_BYTES +
                             static_cast<uint32_t>(kl) * 128u;
     const uint32_t sw = static_cast<uint32_t>(kl & 7);
     const uint64_t c1x2 = f2_pack(p.c1, p.c1);
-    // Row terms of iteration i for this lane's row (loaded one iteration ahead by the stager).
-    auto row_terms = [&](int it, float& na, float& nd) {
-      na = 0.f;
-      nd = 0.f;
-      if (!stager || it >= n_iter) return;
+    // Row terms of iteration it into L1 (two 128-byte lines each of na and nd for the chunk's
+    // 32 rows), so the broadcast loads of the elementwise steps hit.
+    auto prefetch_terms = [&](int it) {
+      if (it >= n_iter || lane >= 4) return;
       const int r = it / nt, i = it0 + it % nt;
-      const int h = g * p.R + r;
-      const int rr = i * 128 + wg * 32 + lane;
-      if (rr < lq) {
-        const size_t li = static_cast<size_t>(h) * p.total_q + q0 + rr;
-        na = -__ldg(p.lse + li) * LOG2E;
-        if constexpr (BIAS == BIAS_LINEAR)
-          na = fmaf(-__ldg(p.slopes + h) * LOG2E, static_cast<float>(lane), na);
-        nd = -p.delta[li];
-      }
+      const size_t w0 = static_cast<size_t>(g * p.R + r) * p.t_pad + q0 + i * 128 + wg * 32;
+      prefetch_l1((lane < 2 ? p.na : p.nd) + w0 + (lane & 1) * 31);
     };
-    float na_n, nd_n;
-    row_terms(0, na_n, nd_n);
+    prefetch_terms(0);
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
-      ok = mbar_wait(TBAR(B_SF), it & 1, abort_flag, tmo, ecode | 5);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
+      prefetch_terms(it + 1);
       const int r = it / nt, i = it0 + it % nt;
       const int h = g * p.R + r;
-      const int row0 = i * 128;
+      const int rc0 = i * 128 + wg * 32;  // first row of this warpgroup's chunk
       float slope2 = 0.f;
       if constexpr (ALIBI) slope2 = __ldg(p.slopes + h) * LOG2E;
-      const int rc0 = row0 + wg * 32;  // first row of this warpgroup's chunk
-      uint32_t sv[16], dv[16];
-      tmem_ld16(t_lane + T_S + wg * 32, sv);
-      tmem_ld16(t_lane + T_DP + wg * 32, dv);
-      // Every warp finished reading the previous staged terms before B_SF (it waits for all
-      // elementwise warps' B_PF), so the stager may overwrite them now.
-      if (stager) {
-        sts_f32(stage + (lane >> 1) * 16u + (lane & 1) * 4u, na_n);
-        sts_f32(stage + (lane >> 1) * 16u + 8u + (lane & 1) * 4u, nd_n);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(TBAR(B_STF + wg));
-        row_terms(it + 1, na_n, nd_n);
-      }
+      // row terms of the chunk's 32 rows (pad rows past the last token keep these in bounds)
+      const size_t wrow = static_cast<size_t>(h) * p.t_pad + q0 + rc0;
+      const float* na_row = p.na + wrow;
+      const float* nd_row = p.nd + wrow;
       // rows rc0 + e with e_lo <= e < e_hi see this key
       const int e_hi = key < lk ? min(32, lq - rc0) : 0;
       const int e_lo = CAUSAL ? key - shift - rc0 : 0;
       const bool full = __all_sync(0xffffffffu, e_lo <= 0 && e_hi >= 32);
       const float dd = static_cast<float>(rc0 + shift - key);
       const uint64_t kb2 = f2_pack(-slope2 * dd, -slope2 * dd);
-      ok = mbar_wait(TBAR(B_STF + wg), it & 1, abort_flag, tmo, ecode | 8);
+      // ---- phase A: P from S^T(i)
+      ok = mbar_wait(TBAR(B_STR), it & 1, abort_flag, tmo, ecode | 5);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      tmem_wait_ld();
-      uint32_t pp[8], pd[8];
-      if (full)
-        bwd_kv_half<BF16, false, BIAS, 0>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, pp, pd);
-      else
-        bwd_kv_half<BF16, true, BIAS, 0>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, pp, pd);
-      tmem_st8(t_lane + T_DP + wg * 32, pd);
-      // The second half of the chunk's S^T / dP^T columns; once it has landed S^T(i) is free.
-      tmem_ld16(t_lane + T_S + wg * 32 + 16, sv);
-      tmem_ld16(t_lane + T_DP + wg * 32 + 16, dv);
+      tc_fence_after();
+      float pr[32];
+      {
+        uint32_t sv[32];
+        tmem_ld32(t_lane + T_S + wg * 32, sv);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(TBAR(B_SE));  // S^T(i) columns free for S^T(i+1)
+        if (full)
+          bwd_kv_p<false, BIAS>(sv, na_row, c1x2, kb2, slope2, dd, e_lo, e_hi, pr);
+        else
+          bwd_kv_p<true, BIAS>(sv, na_row, c1x2, kb2, slope2, dd, e_lo, e_hi, pr);
+      }
+      // ---- phase B: dS from dP^T(i), packed over the chunk's first 16 dP^T columns
+      ok = mbar_wait(TBAR(B_SF), it & 1, abort_flag, tmo, ecode | 8);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        uint32_t dv[16], pd[8];
+        tmem_ld16(t_lane + T_DP + wg * 32, dv);
+        tmem_wait_ld();
+        bwd_kv_ds<BF16, 0>(pr, dv, nd_row, pd);
+        tmem_st8(t_lane + T_DP + wg * 32, pd);
+        tmem_ld16(t_lane + T_DP + wg * 32 + 16, dv);  // columns the store above did not touch
+        tmem_wait_ld();
+        bwd_kv_ds<BF16, 1>(pr, dv, nd_row, pd);
+        tmem_st8(t_lane + T_DP + wg * 32 + 8, pd);
+      }
       // P^T(i-1) has been read by dV(i-1) before P^T(i) goes over it.
       ok = mbar_wait(TBAR(B_PTE), (it - 1) & 1, abort_flag, tmo, ecode | 9);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + 0) ^ sw) << 4), pp[0], pp[1],
-                   pp[2], pp[3]);
-      st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + 1) ^ sw) << 4), pp[4], pp[5],
-                   pp[6], pp[7]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(TBAR(B_SE));
-      if (full)
-        bwd_kv_half<BF16, false, BIAS, 1>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, pp, pd);
-      else
-        bwd_kv_half<BF16, true, BIAS, 1>(sv, dv, stage, c1x2, kb2, slope2, dd, e_lo, e_hi, pp, pd);
-      tmem_st8(t_lane + T_DP + wg * 32 + 8, pd);
-      st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + 2) ^ sw) << 4), pp[0], pp[1],
-                   pp[2], pp[3]);
-      st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + 3) ^ sw) << 4), pp[4], pp[5],
-                   pp[6], pp[7]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        st_shared_v4(pt_row + ((static_cast<uint32_t>(4 * (wg & 1) + u) ^ sw) << 4),
+                     bpack2<BF16>(pr[8 * u], pr[8 * u + 1]),
+                     bpack2<BF16>(pr[8 * u + 2], pr[8 * u + 3]),
+                     bpack2<BF16>(pr[8 * u + 4], pr[8 * u + 5]),
+                     bpack2<BF16>(pr[8 * u + 6], pr[8 * u + 7]));
       // dS^T in TMEM and P^T in shared memory (generic proxy) reach the tensor core's reads.
       tmem_wait_st();
       fence_proxy_async_smem();
@@ -714,7 +717,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const size_t li = static_cast<size_t>(h) * p.total_q + q0 + row;
     const float lse2 = row < lq ? __ldg(p.lse + li) * LOG2E : 0.f;
-    const float dl = row < lq ? p.delta[li] : 0.f;
+    const float dl = row < lq ? -p.nd[static_cast<size_t>(h) * p.t_pad + q0 + row] : 0.f;
     float slope2 = 0.f;
     if constexpr (ALIBI) slope2 = __ldg(p.slopes + h) * LOG2E;
     constexpr int BIAS = !ALIBI ? BIAS_NONE : (CAUSAL ? BIAS_LINEAR : BIAS_ABS);

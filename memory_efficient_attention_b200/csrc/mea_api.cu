@@ -317,7 +317,7 @@ int launch_bwd_t(const BwdMaps& m, const mea::BwdParams& p, int max_q, int max_k
     return MEA_ERR_CUDA;
   clear_stale_launch_error();
   const unsigned long long tmo = g_timeout_ns.load();
-  const long long rows = static_cast<long long>(p.total_q) * p.hq;
+  const long long rows = static_cast<long long>(p.t_pad) * p.hq;
   if (rows > 0)
     mea::mea_bwd_pre_kernel<D, BF16><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(p);
   if (max_k > 0)
@@ -628,7 +628,8 @@ int mea_wait_selftest(unsigned long long timeout_ns, int arrive, void* stream) {
 
 size_t mea_backward_workspace_size(int total_q, int n_heads_q) {
   if (total_q < 0 || n_heads_q < 1) return 0;
-  return static_cast<size_t>(total_q) * static_cast<size_t>(n_heads_q) * sizeof(float) + 256;
+  return 2 * (static_cast<size_t>(total_q) + 128) * static_cast<size_t>(n_heads_q) *
+             sizeof(float) + 256;
 }
 
 int mea_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
@@ -670,7 +671,10 @@ int mea_backward(const void* q, const void* k, const void* v, const void* out, c
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
-  p.delta = static_cast<float*>(workspace);
+  p.t_pad = total_q + 128;
+  p.nd = static_cast<float*>(workspace);
+  p.na = p.nd + static_cast<size_t>(p.t_pad) * n_heads_q;
+  p.lin_bias = (alibi_slopes != nullptr && mask_kind == MEA_MASK_CAUSAL) ? 1 : 0;
   p.cu_q = cu_seqlens_q;
   p.cu_k = cu_seqlens_k;
   p.slopes = alibi_slopes;

@@ -193,6 +193,11 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// L1 prefetch of the line holding addr (a hint).
+__device__ __forceinline__ void prefetch_l1(const void* addr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(addr));
+}
+
 // L2 prefetch of one tiled box: a hint (no shared memory, no completion to wait for).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const void* desc, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
