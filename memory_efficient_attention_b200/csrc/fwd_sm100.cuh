@@ -569,6 +569,7 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       uint32_t kv_cnt = 0, q_cnt = 0, it_cnt = 0;
       bool ok = true;
+      const uint64_t pol_once = l2_policy_evict_first(), pol_reuse = l2_policy_evict_last();
       FwdWalk w;
       fwd_walk_init(p, w, ranked, s_np);
       int seg = 0, pair = 0, hb = 0;
@@ -594,13 +595,15 @@ __global__ void __launch_bounds__(384, 1)
           ok = mbar_wait(BAR(B_QE), (q_cnt & 1u) ^ 1u, abort_flag, tmo, ecode | 1);
           if (!ok) break;
           mbar_arrive_expect_tx(BAR(B_QF), 2 * C::TILE_BYTES);
+          // Q is read by this item alone: evict-first, so that the K/V tiles that the other
+          // items of the segment read again stay in L2 (evict-last below).
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int a = 0; a < C::ATOMS; ++a)
-              tma_load_3d(q_s + h * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_q, BAR(B_QF),
-                          a * C::ATOM_COLS, cur.hb << p.log2_p,
-                          cur.q0 + cur.tok0 + h * p.tok_per_tile);
+              tma_load_3d_hint(q_s + h * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_q, BAR(B_QF),
+                               a * C::ATOM_COLS, cur.hb << p.log2_p,
+                               cur.q0 + cur.tok0 + h * p.tok_per_tile, pol_once);
           ++q_cnt;
           for (int j = 0; j < nmax && ok; ++j) {
 #pragma unroll 1
@@ -613,8 +616,8 @@ __global__ void __launch_bounds__(384, 1)
               const uint32_t dst = kv_s0 + s * C::TILE_BYTES;
 #pragma unroll
               for (int a = 0; a < C::ATOMS; ++a)
-                tma_load_3d(dst + a * C::ATOM_BYTES, kv ? &tm_v : &tm_k, BAR(B_KVF + s),
-                            a * C::ATOM_COLS, g, cur.k0 + (nmax - 1 - j) * 128);
+                tma_load_3d_hint(dst + a * C::ATOM_BYTES, kv ? &tm_v : &tm_k, BAR(B_KVF + s),
+                                 a * C::ATOM_COLS, g, cur.k0 + (nmax - 1 - j) * 128, pol_reuse);
               ++kv_cnt;
             }
           }
@@ -763,6 +766,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t t_s = t_lane + h * 128;
     const uint32_t t_o = t_lane + C::TM_O + h * D;
     const uint32_t stg = sbase + C::SMEM_STG + static_cast<uint32_t>(warp) * C::STG_WARP;
+    const uint64_t pol_once = l2_policy_evict_first();  // out is written once
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr float LN2 = 0.6931471805599453f;
     uint32_t tile = 0, ocnt = 0, it_cnt = 0;
@@ -874,7 +878,7 @@ __global__ void __launch_bounds__(384, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tm_o, stg, a * 64, c_head, c_tok);
+            tma_store_3d_hint(&tm_o, stg, a * 64, c_head, c_tok, pol_once);
             bulk_commit();
           }
         }
