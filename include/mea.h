@@ -188,7 +188,8 @@ int mea_forward_fp8(const void* q, const void* k, const void* v, void* out, floa
 /*
  * mea_backward_workspace_size — bytes of workspace mea_backward needs: two fp32 per (query
  * head, query token) and per each of 128 pad rows a head (delta = rowsum(dout * out) and the
- * row's exponent term, computed by the first kernel), plus 256 bytes of alignment slack.
+ * row's exponent term, computed by the first kernel), 4096 bytes for the segments' launch
+ * order, plus 256 bytes of alignment slack.
  */
 size_t mea_backward_workspace_size(int total_q, int n_heads_q);
 

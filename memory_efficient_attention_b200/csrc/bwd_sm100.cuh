@@ -8,6 +8,9 @@
 //                        t - q0 the row's index in its segment), both fp32 in the workspace.
 //                        128 zero rows per head follow the last token, so the tile loops of
 //                        the dK/dV kernel may read row terms up to a tile past a segment's end.
+//                        Its first block also ranks the segments by decreasing lq + lk (up to
+//                        kBwdOrderMax of them): the two main kernels launch the segments in
+//                        that order, so the heaviest CTAs start first instead of forming a tail.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -31,6 +34,7 @@ struct BwdParams {
   float* na;            // [Hq, t_pad] workspace: the row's exponent term (see the pre kernel)
   int t_pad;            // total_q + 128
   int lin_bias;         // causal ALiBi: na carries -slope log2 e ((t - q0) mod 32)
+  int* order;           // [n_seqs] workspace: segments by decreasing lq + lk, or null (identity)
   const int32_t* cu_q;
   const int32_t* cu_k;
   const float* slopes;  // [Hq] natural-log ALiBi slopes, or null
@@ -46,8 +50,26 @@ struct BwdParams {
 };
 
 // ------------------------------------------------------------------------------------------
+constexpr int kBwdOrderMax = 1024;
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(128) mea_bwd_pre_kernel(const BwdParams p) {
+  if (blockIdx.x == 0 && p.order) {
+    // rank of segment i = number of segments heavier than it (ties by index): a stable sort
+    __shared__ int len[kBwdOrderMax];
+    for (int i = threadIdx.x; i < p.n_seqs; i += blockDim.x)
+      len[i] = (__ldg(p.cu_q + i + 1) - __ldg(p.cu_q + i)) + (__ldg(p.cu_k + i + 1) - __ldg(p.cu_k + i));
+    __syncthreads();
+    for (int i = threadIdx.x; i < p.n_seqs; i += blockDim.x) {
+      const int li = len[i];
+      int r = 0;
+      for (int j = 0; j < p.n_seqs; ++j) {
+        const int lj = len[j];
+        r += (lj > li || (lj == li && j < i)) ? 1 : 0;
+      }
+      p.order[r] = i;
+    }
+  }
   const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= static_cast<long long>(p.t_pad) * p.hq) return;

@@ -196,7 +196,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   using L = BwdKvCfg<D>;
   static_assert(C::NWG == 4, "one 32-row chunk per elementwise warpgroup");
   constexpr float LOG2E = 1.4426950408889634f;
-  const int jt = blockIdx.x, s = blockIdx.y, g = blockIdx.z;
+  // segments in decreasing order of work (the pre kernel's ranking), key tiles heaviest first
+  const int jt = blockIdx.x, s = p.order ? p.order[blockIdx.y] : blockIdx.y, g = blockIdx.z;
   const int q0 = __ldg(p.cu_q + s), lq = __ldg(p.cu_q + s + 1) - q0;
   const int k0 = __ldg(p.cu_k + s), lk = __ldg(p.cu_k + s + 1) - k0;
   const int key0 = jt * 128;
@@ -551,7 +552,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   // Causal: the last query tiles see the most keys; start them first.
   const int itile = CAUSAL ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
                            : static_cast<int>(blockIdx.x);
-  const int s = blockIdx.y, h = blockIdx.z, g = h / p.R;
+  const int s = p.order ? p.order[blockIdx.y] : blockIdx.y, h = blockIdx.z, g = h / p.R;
   const int q0 = __ldg(p.cu_q + s), lq = __ldg(p.cu_q + s + 1) - q0;
   const int k0 = __ldg(p.cu_k + s), lk = __ldg(p.cu_k + s + 1) - k0;
   const int row0 = itile * 128;

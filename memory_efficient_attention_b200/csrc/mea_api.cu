@@ -629,7 +629,7 @@ int mea_wait_selftest(unsigned long long timeout_ns, int arrive, void* stream) {
 size_t mea_backward_workspace_size(int total_q, int n_heads_q) {
   if (total_q < 0 || n_heads_q < 1) return 0;
   return 2 * (static_cast<size_t>(total_q) + 128) * static_cast<size_t>(n_heads_q) *
-             sizeof(float) + 256;
+             sizeof(float) + mea::kBwdOrderMax * sizeof(int) + 256;
 }
 
 int mea_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
@@ -675,6 +675,9 @@ int mea_backward(const void* q, const void* k, const void* v, const void* out, c
   p.nd = static_cast<float*>(workspace);
   p.na = p.nd + static_cast<size_t>(p.t_pad) * n_heads_q;
   p.lin_bias = (alibi_slopes != nullptr && mask_kind == MEA_MASK_CAUSAL) ? 1 : 0;
+  p.order = n_seqs <= mea::kBwdOrderMax
+                ? reinterpret_cast<int*>(p.na + static_cast<size_t>(p.t_pad) * n_heads_q)
+                : nullptr;
   p.cu_q = cu_seqlens_q;
   p.cu_k = cu_seqlens_k;
   p.slopes = alibi_slopes;

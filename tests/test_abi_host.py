@@ -166,8 +166,8 @@ def test_backward_rejects(lib, kw, rc):
 
 
 def test_backward_workspace_size(lib):
-    assert lib.mea_backward_workspace_size(100, 8) == 2 * (100 + 128) * 8 * 4 + 256
-    assert lib.mea_backward_workspace_size(0, 8) == 2 * 128 * 8 * 4 + 256
+    assert lib.mea_backward_workspace_size(100, 8) == 2 * (100 + 128) * 8 * 4 + 4096 + 256
+    assert lib.mea_backward_workspace_size(0, 8) == 2 * 128 * 8 * 4 + 4096 + 256
     assert lib.mea_backward_workspace_size(-1, 8) == 0
     assert lib.mea_backward_workspace_size(10, 0) == 0
 
