@@ -590,7 +590,8 @@ def run_ours(args, world, rank, local):
                     "value": aggregate_throughput(flops3, world, l3ms) / 1e12,
                     "unit": "TFLOP/s", "ms_per_call": l3ms,
                     "roofline": {"bound": "tensor", "achieved": l3tf, "peak": peak3,
-                                 "unit": "TFLOP/s", "frac": l3tf / peak3, "traffic": None,
+                                 "unit": "TFLOP/s", "frac": l3tf / peak3,
+                                 "traffic": traffic_for("mea_fwd_sm100_kernel_long"),
                                  "peak_kind": "bf16 burst",
                                  "kernel": "mea_fwd_sm100_kernel<128, bf16, causal>",
                                  "flops_per_launch": flops3}}
