@@ -173,3 +173,20 @@ def test_backward_is_deterministic():
     _, b = _run([300, 129], [300, 129], 8, 2, 128, torch.bfloat16, True, True, 0.09, 990)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_backward_many_segments_ranked_with_ties():
+    """300 segments with repeated lengths: the pre kernel ranks them (ties by index) and the
+    dK/dV and dQ grids launch them in that order."""
+    import random
+    rnd = random.Random(4242)
+    lens = [rnd.choice([1, 17, 64, 65, 130, 200]) for _ in range(300)]
+    _check(lens, lens, 4, 2, 64, torch.bfloat16, True, True, 0.125, 4242)
+
+
+def test_backward_more_segments_than_ranked():
+    """1100 segments (beyond the 1024 the pre kernel ranks): launched in index order."""
+    import random
+    rnd = random.Random(4343)
+    lens = [rnd.randint(1, 6) for _ in range(1100)]
+    _check(lens, lens, 2, 1, 32, torch.bfloat16, True, False, 0.2, 4343)

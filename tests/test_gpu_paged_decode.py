@@ -96,6 +96,15 @@ def test_paged_decode_dtypes_dims_alibi(d, dtype, alibi):
     _check([33, 250, 129, 7], 8, 8, d, dtype, 16, alibi, 0.1, 1200)
 
 
+@pytest.mark.parametrize("d", [64, 96, 256])
+@pytest.mark.parametrize("bs", [32, 64, 128])
+def test_paged_decode_dims_block_sizes(d, bs):
+    # head dims 64 and 256 take one 5-D box per block (32 or 64 rows of every atom); 96 the
+    # per-atom 4-D boxes
+    _check([1, 31, 32, 33, 200, 700], 16, 2, d, torch.bfloat16, bs, True, 1 / math.sqrt(d),
+           1300 + d + bs)
+
+
 @pytest.mark.parametrize("split", [64, 128, 512])
 def test_paged_decode_explicit_chunks(split):
     _check([2000, 70, 1, 513], 64, 8, 128, torch.bfloat16, 16, True, 0.088, 1300, split)
