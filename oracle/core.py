@@ -26,7 +26,7 @@ Sources (the pages, cited by title and section):
 * [zizhi §1] "大模型推理加速终极指南：xformers如何让Transformer性能飙升300%", section 1
   "分块注意力计算引擎": blockwise computation, split-K attention over the key axis.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (each one is a choice of this implementation):
 
 * causal alignment when L_q != L_k is bottom-right: query row i of a segment sits at key
   position ``p_i = i + L_k - L_q`` (parity unpinned except for L_q = L_k and L_q = 1);
