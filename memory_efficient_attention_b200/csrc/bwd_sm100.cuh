@@ -2,8 +2,8 @@
 //
 // The backward computes dq, dk, dv of L = sum(out * dout) for the forward's definition; its
 // main kernels (tcgen05) are in bwd_tc_sm100.cuh. This file holds the parameter block and
-//   mea_bwd_pre_kernel   per (query head, token) row, one warp each (HBM-bound: reads out and
-//                        dout once): nd = -rowsum(dO * O) = -delta and the row's exponent term
+//   mea_bwd_pre_kernel   per (query head, token) row, one warp per token over its heads
+//                        (HBM-bound: reads out and dout once): nd = -rowsum(dO * O) = -delta and the row's exponent term
 //                        na = -lse log2 e (causal ALiBi: also - slope log2 e ((t - q0) mod 32),
 //                        t - q0 the row's index in its segment), both fp32 in the workspace.
 //                        128 zero rows per head follow the last token, so the tile loops of
@@ -70,57 +70,61 @@ __global__ void __launch_bounds__(128) mea_bwd_pre_kernel(const BwdParams p) {
       p.order[r] = i;
     }
   }
-  const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  // One warp per token (four per block): the token's segment is found once, and the rows of
+  // its heads, adjacent in memory, are read by the lanes together.
+  const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= static_cast<long long>(p.t_pad) * p.hq) return;
-  const int t = static_cast<int>(row / p.hq), h = static_cast<int>(row % p.hq);
-  const size_t wi = static_cast<size_t>(h) * p.t_pad + t;
-  if (t >= p.total_q) {  // pad row
-    if (lane == 0) {
-      p.nd[wi] = 0.f;
-      p.na[wi] = 0.f;
+  if (t >= p.t_pad) return;
+  if (t >= p.total_q) {  // pad rows
+    for (int h = lane; h < p.hq; h += 32) {
+      p.nd[static_cast<size_t>(h) * p.t_pad + t] = 0.f;
+      p.na[static_cast<size_t>(h) * p.t_pad + t] = 0.f;
     }
     return;
   }
-  // lane takes the element pairs 2*lane + 64*i of the row's dh (even) elements
-  const size_t base = (static_cast<size_t>(t) * p.hq + h) * p.dh;
-  const uint16_t* o = reinterpret_cast<const uint16_t*>(p.out) + base;
-  const uint16_t* g = reinterpret_cast<const uint16_t*>(p.dout) + base;
-  float acc = 0.f;
-#pragma unroll
-  for (int i = 0; i < (D + 63) / 64; ++i) {
-    const int e = 64 * i + 2 * lane;
-    if (e >= p.dh) break;
-    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + e);
-    const uint32_t gv = *reinterpret_cast<const uint32_t*>(g + e);
-    float o0, o1, g0, g1;
-    if constexpr (BF16) {
-      const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov));
-      const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv));
-      o0 = of.x; o1 = of.y; g0 = gf.x; g1 = gf.y;
-    } else {
-      const float2 of = __half22float2(*reinterpret_cast<const __half2*>(&ov));
-      const float2 gf = __half22float2(*reinterpret_cast<const __half2*>(&gv));
-      o0 = of.x; o1 = of.y; g0 = gf.x; g1 = gf.y;
-    }
-    acc = fmaf(o0, g0, acc);
-    acc = fmaf(o1, g1, acc);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    constexpr float LOG2E = 1.4426950408889634f;
-    float na = -__ldg(p.lse + static_cast<size_t>(h) * p.total_q + t) * LOG2E;
-    if (p.lin_bias) {
+  constexpr float LOG2E = 1.4426950408889634f;
+  int e_row = 0;  // the token's index in its segment, mod 32 (causal ALiBi only)
+  if (p.lin_bias) {
+    if (lane == 0) {
       // start of the token's segment: the last s with cu_q[s] <= t
       int lo = 0, hi = p.n_seqs;
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (__ldg(p.cu_q + mid) <= t) lo = mid; else hi = mid;
       }
-      const int e = (t - __ldg(p.cu_q + lo)) & 31;
-      na = fmaf(-__ldg(p.slopes + h) * LOG2E, static_cast<float>(e), na);
+      e_row = (t - __ldg(p.cu_q + lo)) & 31;
     }
+    e_row = __shfl_sync(0xffffffffu, e_row, 0);
+  }
+  // Lane h takes head h (and h + 32, ...): the whole row dot product from 16-byte read-only
+  // loads, so that every head's row of the token is in flight at once.
+  for (int h = lane; h < p.hq; h += 32) {
+    const size_t base = (static_cast<size_t>(t) * p.hq + h) * p.dh;
+    const uint4* o4 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.out) + base);
+    const uint4* g4 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + base);
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      if (c * 8 >= p.dh) break;
+      const uint4 ov = __ldg(o4 + c), gv = __ldg(g4 + c);
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float2 of, gf;
+        if constexpr (BF16) {
+          of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[u]));
+          gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[u]));
+        } else {
+          of = __half22float2(*reinterpret_cast<const __half2*>(&ow[u]));
+          gf = __half22float2(*reinterpret_cast<const __half2*>(&gw[u]));
+        }
+        acc = fmaf(of.x, gf.x, acc);
+        acc = fmaf(of.y, gf.y, acc);
+      }
+    }
+    const size_t wi = static_cast<size_t>(h) * p.t_pad + t;
+    float na = -__ldg(p.lse + static_cast<size_t>(h) * p.total_q + t) * LOG2E;
+    if (p.lin_bias) na = fmaf(-__ldg(p.slopes + h) * LOG2E, static_cast<float>(e_row), na);
     p.nd[wi] = -acc;
     p.na[wi] = na;
   }

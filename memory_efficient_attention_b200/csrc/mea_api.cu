@@ -317,9 +317,8 @@ int launch_bwd_t(const BwdMaps& m, const mea::BwdParams& p, int max_q, int max_k
     return MEA_ERR_CUDA;
   clear_stale_launch_error();
   const unsigned long long tmo = g_timeout_ns.load();
-  const long long rows = static_cast<long long>(p.t_pad) * p.hq;
-  if (rows > 0)
-    mea::mea_bwd_pre_kernel<D, BF16><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(p);
+  // one warp per token (including the pad rows), four per block
+  mea::mea_bwd_pre_kernel<D, BF16><<<static_cast<unsigned>((p.t_pad + 3) / 4), 128, 0, stream>>>(p);
   if (max_k > 0)
     kdkdv<<<dim3((max_k + 127) / 128, p.n_seqs, p.hkv), mea::BwdTcCfg<D>::THREADS, smem,
             stream>>>(m.q, m.dout, m.k, m.v, p, tmo);
