@@ -207,7 +207,8 @@ size_t mea_backward_workspace_size(int total_q, int n_heads_q);
  *   dq, dk, dv    DEVICE outputs, layouts of q, k, v; every element is written (keys no query
  *                 sees and rows that see no key get 0).
  *   n_seqs        1 .. 65535 segments.
- *   max_seqlen_q/k upper bounds on every L_q / L_k (they size the grids).
+ *   max_seqlen_q/k upper bounds on every L_q / L_k (they size the grids; MEA_ERR_SHAPE when
+ *                 ceil(max_seqlen_q / 128) * n_heads_q / 4 would pass 2^31 - 1).
  *   workspace     DEVICE, at least mea_backward_workspace_size(total_q, n_heads_q) bytes, owned
  *                 by the caller; 16-byte aligned.
  * No atomics: the result is deterministic. Asynchronous on `stream`. Returns MEA_OK or a

@@ -45,6 +45,7 @@ struct BwdParams {
   int hkv;
   int dh;               // head dim of the rows (<= D; the TMA zero-fills the columns past it)
   int R;                // query heads per KV head
+  int mq;               // query heads per dQ CTA (divides hq)
   float scale;
   float c1;             // scale * log2(e)
 };

@@ -19,10 +19,12 @@
 // over the whole GQA group; they are written once. Since P^T does not sit in TMEM, S^T(i+1) is
 // computed while the elementwise warps still work on iteration i.
 //
-// mea_bwd_dq_tc_kernel: one CTA per (128-row query tile, segment, query head), over the key
-// tiles the rows see: S = Q K^T, dP = dO V^T, dS (thread = row), dQ += dS K.
-// TMEM: S(j) in [0,128) or [128,256) by the parity of j, dP [256,384), dQ [384,384+D); S(j+2)
-// is computed while the elementwise warps work on tile j+1.
+// mea_bwd_dq_tc_kernel: one CTA per (128-row query tile, segment, group of mq query heads);
+// for each head in turn (an item), over the key tiles the rows see: S = Q K^T, dP = dO V^T, dS
+// (thread = row), dQ += dS K. TMEM: S(j) in [0,128) or [128,256) by the parity of j (counted over
+// the CTA's items), dP [256,384), dQ [384,384+D); S(j+2) is computed while the elementwise warps
+// work on tile j+1, and the next item's Q/dO load and first S/dP overlap the current item's last
+// tile and the read-out of its dQ.
 //
 // Roles (NWG*128 + 64 threads): NWG elementwise warpgroups (thread = TMEM lane; group w handles
 // the 32-column chunks [128w/NWG, 128(w+1)/NWG) of the S/dP tiles and writes its packed P / dS
@@ -340,7 +342,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       for (int it = 0; it < n_iter && ok; ++it) {
         if (it + 1 < n_iter) {
           // ---- S^T(i+1) = K Q(i+1)^T into the columns S^T(i) was read from
-          ok = mbar_wait(TBAR(B_QF + ((it + 1) & 1)), ((it + 1) >> 1) & 1, abort_flag, tmo,
+          ok = mbar_wait_fast(TBAR(B_QF + ((it + 1) & 1)), ((it + 1) >> 1) & 1, abort_flag, tmo,
                          ecode | 3);
           if (ok) ok = mbar_wait_spin(TBAR(B_SE), it & 1, abort_flag, tmo, ecode | 7);
           if (!ok) break;
@@ -361,7 +363,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
         mma_commit(TBAR(B_QE + (it & 1)));
         // ---- dP^T(i+1) = V dO(i+1)^T over the dS^T(i) columns dK has just read
         if (it + 1 < n_iter) {
-          ok = mbar_wait(TBAR(B_DF + ((it + 1) & 1)), ((it + 1) >> 1) & 1, abort_flag, tmo,
+          ok = mbar_wait_fast(TBAR(B_DF + ((it + 1) & 1)), ((it + 1) >> 1) & 1, abort_flag, tmo,
                          ecode | 3);
           if (!ok) break;
           tc_fence_after();
@@ -526,8 +528,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
 }
 
 // -------------------------------------------------------------------------------------------
-// dQ kernel layout: Q and dO loaded once; K in a 3-stage ring (its last use, dQ(j), comes a tile
-// after S(j+2) would like to reuse the stage), V in a 2-stage ring (free after dP(j)).
+// dQ kernel layout: Q and dO of the current item; K in a 3-stage ring (its last use, dQ(j), comes
+// a tile after S(j+2) would like to reuse the stage), V in a 2-stage ring (free after dP(j)).
 template <int D>
 struct BwdDqCfg {
   using T = BwdTcCfg<D>;
@@ -539,6 +541,8 @@ struct BwdDqCfg {
   static_assert(SMEM_TOTAL <= 232448, "shared memory per CTA");
 };
 
+// Grid: x = query tile * (hq / mq) + group of mq query heads (causal: the last tiles, which see
+// the most keys, first), y = segment in the pre kernel's order (heaviest first).
 template <int D, bool BF16, bool CAUSAL, bool ALIBI>
 __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     mea_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -549,24 +553,28 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   using C = BwdTcCfg<D>;
   using L = BwdDqCfg<D>;
   constexpr float LOG2E = 1.4426950408889634f;
-  // Causal: the last query tiles see the most keys; start them first.
-  const int itile = CAUSAL ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
-                           : static_cast<int>(blockIdx.x);
-  const int s = p.order ? p.order[blockIdx.y] : blockIdx.y, h = blockIdx.z, g = h / p.R;
+  const int n_grp = p.hq / p.mq, bx = static_cast<int>(blockIdx.x);
+  const int n_tiles = static_cast<int>(gridDim.x) / n_grp, tl = bx / n_grp;
+  const int itile = CAUSAL ? n_tiles - 1 - tl : tl;
+  const int s = p.order ? p.order[blockIdx.y] : blockIdx.y;
+  const int h0 = (bx - tl * n_grp) * p.mq, n_items = p.mq;
   const int q0 = __ldg(p.cu_q + s), lq = __ldg(p.cu_q + s + 1) - q0;
   const int k0 = __ldg(p.cu_k + s), lk = __ldg(p.cu_k + s + 1) - k0;
   const int row0 = itile * 128;
-  if (row0 >= lq) return;
+  if (row0 >= lq) return;  // the whole CTA leaves before any shared state exists
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sb = smem_u32(smem);
-  // B_KF/B_KE: K ring (3), B_VF/B_VE: V ring (2); B_SF: S(j) and dP(j) in TMEM; B_PF: dS(j)
-  // packed by the elementwise warps (dP free again).
-  constexpr int B_QD = 0, B_KF = 1, B_KE = 4, B_VF = 7, B_VE = 9, B_SF = 11, B_PF = 12,
-                B_ACC = 13, B_DR = 14;
-  constexpr int N_BARS = 15;
+  // Per tile (gt counts tiles over the CTA's items): B_KF/B_KE the K ring (3), B_VF/B_VE the V
+  // ring (2), B_SF S(gt) and dP(gt) in TMEM, B_PF dS(gt) packed by the elementwise warps. Per item
+  // (m): B_QF/B_QE Q and dO loaded / no longer read, B_ACC dQ complete, B_DQE dQ read out of TMEM
+  // by the elementwise warps (the next item may accumulate over it).
+  constexpr int B_QF = 0, B_KF = 1, B_KE = 4, B_VF = 7, B_VE = 9, B_SF = 11, B_PF = 12,
+                B_ACC = 13, B_DR = 14, B_QE = 15, B_DQE = 16;
+  constexpr int N_BARS = 17;
+  static_assert(8 * N_BARS + 8 <= 256, "barrier area");
   const uint32_t bar0 = sb + L::SMEM_BAR;
 #define TBAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SMEM_BAR + 8 * N_BARS);
@@ -575,6 +583,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   const unsigned ecode = (KID_BWD << 8) | 0x80;
   const uint64_t tmo = timeout_ns;
 
+  // Every item of the CTA covers the same rows, hence the same key tiles.
   const int shift = lk - lq;
   const int nrows = min(128, lq - row0);
   int n_jt = (lk + 127) / 128;
@@ -584,7 +593,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(TBAR(B_QD), 1);
+    mbar_init(TBAR(B_QF), 1);
+    mbar_init(TBAR(B_QE), 1);
     for (int b = 0; b < 3; ++b) {
       mbar_init(TBAR(B_KF + b), 1);
       mbar_init(TBAR(B_KE + b), 1);
@@ -594,9 +604,10 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       mbar_init(TBAR(B_VE + b), 1);
     }
     mbar_init(TBAR(B_SF), 1);
-    mbar_init(TBAR(B_PF), 4 * C::NWG);  // one elected arrival per elementwise warp
+    mbar_init(TBAR(B_PF), 4 * C::NWG);   // one elected arrival per elementwise warp
     mbar_init(TBAR(B_ACC), 1);
     mbar_init(TBAR(B_DR), 1);
+    mbar_init(TBAR(B_DQE), 4 * C::NWG);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -608,72 +619,89 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM: S(j) in buffer j mod 2, then dP and the dQ accumulator.
+  // TMEM: S(gt) in buffer gt mod 2, then dP and the dQ accumulator.
   const uint32_t T_S0 = 0, T_DP = 256, T_DQ = 384;
 
   if (warp == C::W_LOAD) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
-      int nk = 0, nv = 0;  // K / V loads issued
-      mbar_arrive_expect_tx(TBAR(B_QD), 2 * C::TILE_BYTES);
-#pragma unroll
-      for (int a = 0; a < C::ATOMS; ++a) {
-        tma_load_3d(sb + L::SMEM_Q + a * C::ATOM_BYTES, &tm_q, TBAR(B_QD), a * 64, h, q0 + row0);
-        tma_load_3d(sb + L::SMEM_DO + a * C::ATOM_BYTES, &tm_do, TBAR(B_QD), a * 64, h,
-                    q0 + row0);
-      }
-      for (int jt = 0; jt < n_jt && ok; ++jt) {
-        const int kb = jt % 3, vb = jt & 1;
-        ok = mbar_wait(TBAR(B_KE + kb), ((jt / 3) & 1) ^ 1, abort_flag, tmo, ecode | 1);
+      uint32_t gk = 0, gv = 0;  // K / V tiles loaded over the CTA's items
+      int nq = 0;               // items whose Q / dO were issued
+      for (int m = 0; m < n_items && ok; ++m) {
+        const int h = h0 + m, g = h / p.R;
+        // Q and dO of item m, once the previous item no longer reads them
+        ok = mbar_wait(TBAR(B_QE), (m & 1) ^ 1, abort_flag, tmo, ecode | 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(TBAR(B_KF + kb), C::TILE_BYTES);
+        if (n_jt > 0) {
+          mbar_arrive_expect_tx(TBAR(B_QF), 2 * C::TILE_BYTES);
 #pragma unroll
-        for (int a = 0; a < C::ATOMS; ++a)
-          tma_load_3d(sb + L::SMEM_K + kb * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_k,
-                      TBAR(B_KF + kb), a * 64, g, k0 + jt * 128);
-        nk = jt + 1;
-        ok = mbar_wait(TBAR(B_VE + vb), ((jt >> 1) & 1) ^ 1, abort_flag, tmo, ecode | 1);
-        if (!ok) break;
-        mbar_arrive_expect_tx(TBAR(B_VF + vb), C::TILE_BYTES);
+          for (int a = 0; a < C::ATOMS; ++a) {
+            tma_load_3d(sb + L::SMEM_Q + a * C::ATOM_BYTES, &tm_q, TBAR(B_QF), a * 64, h,
+                        q0 + row0);
+            tma_load_3d(sb + L::SMEM_DO + a * C::ATOM_BYTES, &tm_do, TBAR(B_QF), a * 64, h,
+                        q0 + row0);
+          }
+        } else {
+          mbar_arrive(TBAR(B_QF));
+        }
+        nq = m + 1;
+        for (int jt = 0; jt < n_jt && ok; ++jt) {
+          const uint32_t kb = gk % 3, vb = gv & 1;
+          ok = mbar_wait(TBAR(B_KE + kb), ((gk / 3) & 1) ^ 1, abort_flag, tmo, ecode | 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(TBAR(B_KF + kb), C::TILE_BYTES);
 #pragma unroll
-        for (int a = 0; a < C::ATOMS; ++a)
-          tma_load_3d(sb + L::SMEM_V + vb * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_v,
-                      TBAR(B_VF + vb), a * 64, g, k0 + jt * 128);
-        nv = jt + 1;
+          for (int a = 0; a < C::ATOMS; ++a)
+            tma_load_3d(sb + L::SMEM_K + kb * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_k,
+                        TBAR(B_KF + kb), a * 64, g, k0 + jt * 128);
+          ++gk;
+          ok = mbar_wait(TBAR(B_VE + vb), ((gv >> 1) & 1) ^ 1, abort_flag, tmo, ecode | 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(TBAR(B_VF + vb), C::TILE_BYTES);
+#pragma unroll
+          for (int a = 0; a < C::ATOMS; ++a)
+            tma_load_3d(sb + L::SMEM_V + vb * C::TILE_BYTES + a * C::ATOM_BYTES, &tm_v,
+                        TBAR(B_VF + vb), a * 64, g, k0 + jt * 128);
+          ++gv;
+        }
       }
       // Let every issued load land before shared memory goes away.
       volatile int never = 0;
-      mbar_wait(TBAR(B_QD), 0, &never, tmo, ecode | 15);
-      for (int jt = max(0, nk - 3); jt < nk; ++jt)
-        mbar_wait(TBAR(B_KF + jt % 3), (jt / 3) & 1, &never, tmo, ecode | 15);
-      for (int jt = max(0, nv - 2); jt < nv; ++jt)
-        mbar_wait(TBAR(B_VF + (jt & 1)), (jt >> 1) & 1, &never, tmo, ecode | 15);
+      if (nq > 0) mbar_wait(TBAR(B_QF), (nq - 1) & 1, &never, tmo, ecode | 15);
+      for (uint32_t x = (gk > 3 ? gk - 3 : 0); x < gk; ++x)
+        mbar_wait(TBAR(B_KF + x % 3), (x / 3) & 1, &never, tmo, ecode | 15);
+      for (uint32_t x = (gv > 2 ? gv - 2 : 0); x < gv; ++x)
+        mbar_wait(TBAR(B_VF + (x & 1)), (x >> 1) & 1, &never, tmo, ecode | 15);
     }
   } else if (warp == C::W_ISSUE) {
     // ------------------------------------------------------------ tcgen05 issuer
-    // Order: S(0), dP(0), S(1); then per tile j, once dS(j) is packed: dP(j+1) (the next
-    // elementwise step can start after this one GEMM), dQ += dS(j) K(j), S(j+2) into the
-    // buffer dQ(j) has just read.
+    // Per item: S(0), dP(0), S(1); then per tile j, once dS(j) is packed: dP(j+1) (the next
+    // elementwise step waits for that one GEMM only, S(j+1) being already there), dQ(j) (the
+    // item's first one waits until the previous item's dQ has been read out of TMEM), then
+    // S(j+2) into the buffer dQ(j) has just read. Once the item's last dP is issued, its Q / dO
+    // go back to the producer, which loads the next item's while this one finishes.
     if (lane == 0) {
       constexpr uint32_t ID_KK = umma_idesc_f16(BF16, 128, 128, false, false);
       constexpr uint32_t ID_PV = umma_idesc_f16(BF16, 128, D, false, true);
-      auto issue_s = [&](int jt) -> bool {
-        const int kb = jt % 3;
-        if (!mbar_wait(TBAR(B_KF + kb), (jt / 3) & 1, abort_flag, tmo, ecode | 3)) return false;
+      auto issue_s = [&](uint32_t gt) -> bool {
+        const uint32_t kb = gt % 3;
+        if (!mbar_wait_fast(TBAR(B_KF + kb), (gt / 3) & 1, abort_flag, tmo, ecode | 3))
+          return false;
         tc_fence_after();
         const uint32_t ks = sb + L::SMEM_K + kb * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + T_S0 + (jt & 1) * 128, umma_desc_sw128(sb + L::SMEM_Q + off, 16, 1024),
+          mma_ss(tmem + T_S0 + (gt & 1) * 128, umma_desc_sw128(sb + L::SMEM_Q + off, 16, 1024),
                  umma_desc_sw128(ks + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
         }
         return true;
       };
-      auto issue_dp = [&](int jt) -> bool {
-        const int vb = jt & 1;
-        if (!mbar_wait(TBAR(B_VF + vb), (jt >> 1) & 1, abort_flag, tmo, ecode | 3)) return false;
+      auto issue_dp = [&](uint32_t gt) -> bool {
+        const uint32_t vb = gt & 1;
+        if (!mbar_wait_fast(TBAR(B_VF + vb), (gt >> 1) & 1, abort_flag, tmo, ecode | 3))
+          return false;
         tc_fence_after();
         const uint32_t vs = sb + L::SMEM_V + vb * C::TILE_BYTES;
 #pragma unroll
@@ -683,29 +711,53 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
                  umma_desc_sw128(vs + off, 16, 1024), ID_KK, kk > 0 ? 1u : 0u);
         }
         mma_commit(TBAR(B_VE + vb));
-        mma_commit(TBAR(B_SF));  // S(j) (issued earlier) and dP(j)
+        mma_commit(TBAR(B_SF));  // S(gt) (issued earlier) and dP(gt)
         return true;
       };
-      bool ok = mbar_wait(TBAR(B_QD), 0, abort_flag, tmo, ecode | 2);
-      tc_fence_after();
-      if (ok && n_jt > 0) ok = issue_s(0) && issue_dp(0);
-      if (ok && n_jt > 1) ok = issue_s(1);
-      for (int jt = 0; jt < n_jt && ok; ++jt) {
-        ok = mbar_wait_spin(TBAR(B_PF), jt & 1, abort_flag, tmo, ecode | 4);
+      bool ok = true;
+      const uint32_t n = static_cast<uint32_t>(n_jt);
+      for (int m = 0; m < n_items && ok; ++m) {
+        const uint32_t g = static_cast<uint32_t>(m) * n;  // tiles of the previous items
+        ok = mbar_wait(TBAR(B_QF), m & 1, abort_flag, tmo, ecode | 2);
         if (!ok) break;
         tc_fence_after();
-        if (jt + 1 < n_jt && !(ok = issue_dp(jt + 1))) break;
-        // ---- dQ += dS(j) K(j)
-        const uint32_t ks = sb + L::SMEM_K + (jt % 3) * C::TILE_BYTES;
+        if (n > 0) {
+          ok = issue_s(g) && issue_dp(g);
+          if (ok && n == 1) mma_commit(TBAR(B_QE));
+          if (ok && n > 1) ok = issue_s(g + 1);
+        } else {
+          // No tiles: B_ACC(m) still waits for the read-out of item m-1, so that the per-item
+          // barriers never run two phases ahead of the elementwise warps.
+          mma_commit(TBAR(B_QE));
+          ok = mbar_wait_spin(TBAR(B_DQE), (m & 1) ^ 1, abort_flag, tmo, ecode | 7);
+        }
+        for (uint32_t jt = 0; jt < n && ok; ++jt) {
+          const uint32_t gt = g + jt;
+          ok = mbar_wait_spin(TBAR(B_PF), gt & 1, abort_flag, tmo, ecode | 4);
+          if (!ok) break;
+          tc_fence_after();
+          if (jt + 1 < n) {
+            if (!(ok = issue_dp(gt + 1))) break;
+            if (jt + 2 == n) mma_commit(TBAR(B_QE));  // the item's last read of Q / dO
+          }
+          if (jt == 0) {
+            // the previous item's dQ has been read out of TMEM
+            ok = mbar_wait_spin(TBAR(B_DQE), (m & 1) ^ 1, abort_flag, tmo, ecode | 7);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          // ---- dQ += dS(j) K(j)
+          const uint32_t ks = sb + L::SMEM_K + (gt % 3) * C::TILE_BYTES;
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          mma_ts(tmem + T_DQ, tmem + T_S0 + (jt & 1) * 128 + C::packed_col(k16),
-                 umma_desc_sw128(ks + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
-                 (jt > 0 || k16 > 0) ? 1u : 0u);
-        mma_commit(TBAR(B_KE + jt % 3));
-        if (jt + 2 < n_jt && !(ok = issue_s(jt + 2))) break;
+          for (int k16 = 0; k16 < 8; ++k16)
+            mma_ts(tmem + T_DQ, tmem + T_S0 + (gt & 1) * 128 + C::packed_col(k16),
+                   umma_desc_sw128(ks + k16 * 2048, C::ATOM_BYTES, 1024), ID_PV,
+                   (jt > 0 || k16 > 0) ? 1u : 0u);
+          mma_commit(TBAR(B_KE + gt % 3));
+          if (jt + 2 < n && !(ok = issue_s(gt + 2))) break;
+        }
+        if (ok) mma_commit(TBAR(B_ACC));
       }
-      mma_commit(TBAR(B_ACC));
       mma_commit(TBAR(B_DR));
       volatile int never = 0;
       mbar_wait(TBAR(B_DR), 0, &never, tmo, ecode | 14);
@@ -716,64 +768,65 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
     const int rl = threadIdx.x & 127;
     const int row = row0 + rl;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const size_t li = static_cast<size_t>(h) * p.total_q + q0 + row;
-    const float lse2 = row < lq ? __ldg(p.lse + li) * LOG2E : 0.f;
-    const float dl = row < lq ? -p.nd[static_cast<size_t>(h) * p.t_pad + q0 + row] : 0.f;
-    float slope2 = 0.f;
-    if constexpr (ALIBI) slope2 = __ldg(p.slopes + h) * LOG2E;
     constexpr int BIAS = !ALIBI ? BIAS_NONE : (CAUSAL ? BIAS_LINEAR : BIAS_ABS);
     const uint64_t c1x2 = f2_pack(p.c1, p.c1);
-    const uint64_t nd2 = f2_pack(-dl, -dl);
+    using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     bool ok = true;
-    for (int jt = 0; jt < n_jt && ok; ++jt) {
-      ok = mbar_wait(TBAR(B_SF), jt & 1, abort_flag, tmo, ecode | 5);
+    for (int m = 0; m < n_items && ok; ++m) {
+      const int h = h0 + m;
+      const uint32_t g = static_cast<uint32_t>(m * n_jt);  // tiles of the previous items
+      const size_t li = static_cast<size_t>(h) * p.total_q + q0 + row;
+      const float lse2 = row < lq ? __ldg(p.lse + li) * LOG2E : 0.f;
+      const float dl = row < lq ? -p.nd[static_cast<size_t>(h) * p.t_pad + q0 + row] : 0.f;
+      float slope2 = 0.f;
+      if constexpr (ALIBI) slope2 = __ldg(p.slopes + h) * LOG2E;
+      const uint64_t nd2 = f2_pack(-dl, -dl);
+      for (int jt = 0; jt < n_jt && ok; ++jt) {
+        const uint32_t gt = g + static_cast<uint32_t>(jt);
+        ok = mbar_wait(TBAR(B_SF), gt & 1, abort_flag, tmo, ecode | 5);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t t_s = T_S0 + (gt & 1) * 128;
+#pragma unroll 1
+        for (int cc = 0; cc < C::CPW; ++cc) {
+          const int c = C::CPW * wg + cc;
+          uint32_t sv[32], dv[32];
+          tmem_ld32(t_lane + t_s + c * 32, sv);
+          tmem_ld32(t_lane + T_DP + c * 32, dv);
+          // keys kc0 + e with e < e_hi are seen by this row
+          const int kc0 = jt * 128 + c * 32;
+          const int dk = row + shift - kc0;
+          int e_hi = row < lq ? min(32, lk - kc0) : 0;
+          if (CAUSAL) e_hi = min(e_hi, dk + 1);
+          const bool full = __all_sync(0xffffffffu, e_hi >= 32);
+          float b = -lse2;
+          if constexpr (BIAS == BIAS_LINEAR) b = fmaf(-slope2, static_cast<float>(dk), b);
+          tmem_wait_ld();
+          const uint32_t t_d = t_lane + t_s + 32 * C::CPW * wg + cc * 16;
+          if (full)
+            bwd_q_chunk<BF16, false, BIAS>(sv, dv, c1x2, b, slope2, static_cast<float>(dk), nd2,
+                                           e_hi, t_d);
+          else
+            bwd_q_chunk<BF16, true, BIAS>(sv, dv, c1x2, b, slope2, static_cast<float>(dk), nd2,
+                                          e_hi, t_d);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(TBAR(B_PF));
+      }
+      if (!ok) break;
+      // ---- dQ out of TMEM, scaled and packed; group w holds chunk w of the D columns (groups
+      // past D/32 hold none)
+      ok = mbar_wait(TBAR(B_ACC), m & 1, abort_flag, tmo, ecode | 6);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t t_s = T_S0 + (jt & 1) * 128;
-#pragma unroll 1
-      for (int cc = 0; cc < C::CPW; ++cc) {
-        const int c = C::CPW * wg + cc;
-        uint32_t sv[32], dv[32];
-        tmem_ld32(t_lane + t_s + c * 32, sv);
-        tmem_ld32(t_lane + T_DP + c * 32, dv);
-        // keys kc0 + e with e < e_hi are seen by this row
-        const int kc0 = jt * 128 + c * 32;
-        const int dk = row + shift - kc0;
-        int e_hi = row < lq ? min(32, lk - kc0) : 0;
-        if (CAUSAL) e_hi = min(e_hi, dk + 1);
-        const bool full = __all_sync(0xffffffffu, e_hi >= 32);
-        float b = -lse2;
-        if constexpr (BIAS == BIAS_LINEAR) b = fmaf(-slope2, static_cast<float>(dk), b);
-        tmem_wait_ld();
-        const uint32_t t_d = t_lane + t_s + 32 * C::CPW * wg + cc * 16;
-        if (full)
-          bwd_q_chunk<BF16, false, BIAS>(sv, dv, c1x2, b, slope2, static_cast<float>(dk), nd2,
-                                         e_hi, t_d);
-        else
-          bwd_q_chunk<BF16, true, BIAS>(sv, dv, c1x2, b, slope2, static_cast<float>(dk), nd2,
-                                        e_hi, t_d);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(TBAR(B_PF));
-    }
-    if (ok) {
-      ok = mbar_wait(TBAR(B_ACC), 0, abort_flag, tmo, ecode | 6);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      tc_fence_after();
-      using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const bool any = n_jt > 0;
-      const size_t o = (static_cast<size_t>(q0 + row) * p.hq + h) * p.dh;
-      // group w writes its share of the D columns of dQ (groups past D/32 write none)
-      constexpr int CHQ = (D / 32) / C::NWG > 0 ? (D / 32) / C::NWG : 1;
-#pragma unroll 1
-      for (int c = wg * CHQ; c < (wg + 1) * CHQ && c < D / 32; ++c) {
+      if (wg < D / 32) {
         uint32_t a[32];
-        tmem_ld32(t_lane + T_DQ + c * 32, a);
+        tmem_ld32(t_lane + T_DQ + wg * 32, a);
         tmem_wait_ld();
         if (row < lq) {
           uint32_t pa[16];
@@ -782,13 +835,18 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
             pa[u] = any ? bpack2<BF16>(__uint_as_float(a[2 * u]) * p.scale,
                                        __uint_as_float(a[2 * u + 1]) * p.scale)
                         : 0u;
-          uint4* dqp = reinterpret_cast<uint4*>(reinterpret_cast<OutT*>(p.dq) + o + c * 32);
+          const size_t o = (static_cast<size_t>(q0 + row) * p.hq + h) * p.dh;
+          uint4* dqp = reinterpret_cast<uint4*>(reinterpret_cast<OutT*>(p.dq) + o + wg * 32);
 #pragma unroll
           for (int u = 0; u < 4; ++u)
-            if (c * 32 + u * 8 < p.dh)
+            if (wg * 32 + u * 8 < p.dh)
               dqp[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
         }
       }
+      // dQ has been read out of TMEM: the next item may accumulate over it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(TBAR(B_DQE));
     }
   }
   tc_fence_before();

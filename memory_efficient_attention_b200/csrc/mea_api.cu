@@ -323,7 +323,8 @@ int launch_bwd_t(const BwdMaps& m, const mea::BwdParams& p, int max_q, int max_k
     kdkdv<<<dim3((max_k + 127) / 128, p.n_seqs, p.hkv), mea::BwdTcCfg<D>::THREADS, smem,
             stream>>>(m.q, m.dout, m.k, m.v, p, tmo);
   if (max_q > 0)
-    kdq<<<dim3((max_q + 127) / 128, p.n_seqs, p.hq), mea::BwdTcCfg<D>::THREADS, smem_dq,
+    kdq<<<dim3(static_cast<unsigned>((p.hq / p.mq) * ((max_q + 127) / 128)), p.n_seqs),
+          mea::BwdTcCfg<D>::THREADS, smem_dq,
           stream>>>(m.q, m.dout, m.k, m.v, p, tmo);
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
@@ -687,6 +688,11 @@ int mea_backward(const void* q, const void* k, const void* v, const void* out, c
   p.hkv = n_heads_kv;
   p.dh = head_dim;
   p.R = n_heads_q / n_heads_kv;
+  // dQ: one CTA runs the same query tile for mq heads in turn (of one KV group when R allows)
+  p.mq = n_heads_q % 4 == 0 ? 4 : (n_heads_q % 2 == 0 ? 2 : 1);
+  const uint64_t dq_ctas =
+      static_cast<uint64_t>(n_heads_q / p.mq) * ((static_cast<uint64_t>(max_seqlen_q) + 127) / 128);
+  if (dq_ctas > 0x7fffffffull) return MEA_ERR_SHAPE;  // the dQ grid's x dimension
   p.scale = scale;
   p.c1 = scale * 1.4426950408889634f;
   BwdMaps m;

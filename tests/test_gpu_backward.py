@@ -118,7 +118,7 @@ def test_backward_small_packed_workload(causal):
     _check(w.seqlens_q, w.seqlens_k, 8, 8, 64, torch.float16, causal, False, w.scale, w.seed)
 
 
-@pytest.mark.parametrize("hq,hkv", [(8, 2), (12, 4), (9, 3), (4, 1)])
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (12, 4), (9, 3), (4, 1), (6, 2)])
 def test_backward_gqa_causal_alibi(hq, hkv):
     _check([130, 77, 300], [130, 77, 300], hq, hkv, 128, torch.bfloat16, True, True,
            1 / math.sqrt(128), 900 + hq)
