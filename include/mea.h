@@ -22,6 +22,8 @@
  *   cu_seqlens_q / cu_seqlens_k: int32 [n_seqs+1] prefix sums of segment lengths, in DEVICE
  *   memory; segment s owns query rows [cu_q[s], cu_q[s+1]) and key rows [cu_k[s], cu_k[s+1]).
  *   Query head h reads key/value head h / R (the repeat_interleave grouping).
+ *   D: a multiple of 8 from 8 to 256 (mea_forward and the decode entry points), from 8 to 128
+ *   (mea_backward); a multiple of 16 from 16 to 128 with e4m3 inputs (mea_forward_fp8).
  *
  * Per segment s with L_q = cu_q[s+1]-cu_q[s], L_k = cu_k[s+1]-cu_k[s], query row i sits at key
  * position p_i = i + L_k - L_q (bottom-right alignment: the last query sees the last key).
@@ -51,7 +53,7 @@ typedef enum {
   MEA_ERR_NULL = -1,          /* a required pointer is NULL                                   */
   MEA_ERR_SHAPE = -2,         /* negative/zero sizes, total or max_seqlen out of range        */
   MEA_ERR_HEADS = -3,         /* n_heads_q % n_heads_kv != 0, or a head count < 1             */
-  MEA_ERR_HEAD_DIM = -4,      /* head_dim not in {64, 128}                                    */
+  MEA_ERR_HEAD_DIM = -4,      /* head_dim outside the entry point's set (see Notation)        */
   MEA_ERR_DTYPE = -5,         /* dtype not MEA_F16 / MEA_BF16                                 */
   MEA_ERR_ALIGN = -6,         /* a tensor base pointer is not 16-byte aligned (TMA needs it)  */
   MEA_ERR_MASK = -7,          /* mask_kind not a mea_mask value                               */
@@ -174,8 +176,8 @@ int mea_decode_splitkv_noalloc(const void* q, const void* k, const void* v, void
  * masks, GQA grouping, ALiBi and scale as mea_forward. Q K^T accumulates in fp32; P is rounded
  * to e4m3 for the P V product (its row sum and lse use the fp32 values); out is written in
  * out_dtype (MEA_BF16 or MEA_F16), lse in fp32 natural log.
- *   q, k, v   DEVICE e4m3 [total_q, n_heads_q, 128] / [total_k, n_heads_kv, 128].
- *   head_dim  128 only (MEA_ERR_HEAD_DIM otherwise).
+ *   q, k, v   DEVICE e4m3 [total_q, n_heads_q, D] / [total_k, n_heads_kv, D].
+ *   head_dim  a multiple of 16 from 16 to 128 (MEA_ERR_HEAD_DIM otherwise).
  * Other arguments, errors and ownership as mea_forward.
  */
 int mea_forward_fp8(const void* q, const void* k, const void* v, void* out, float* lse,
