@@ -19,7 +19,7 @@ import torch
 
 import memory_efficient_attention_b200 as mea
 import oracle
-from mea_workloads import alibi_slope_values, cu_seqlens, randn
+from mea_workloads import alibi_slope_values, cu_seqlens, randn, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -31,7 +31,8 @@ def _quantized(shape, seed, descale):
     return x.to(torch.float8_e4m3fn)
 
 
-def _case(seqlens, hq, hkv, causal, alibi, scale, seed, out_dtype=torch.bfloat16, d=128):
+def _run(seqlens, hq, hkv, causal, alibi, scale, seed, out_dtype=torch.bfloat16, d=128):
+    """The kernel on seeded e4m3 inputs; returns the host e4m3 codes, the slopes and out, lse."""
     tq = sum(seqlens)
     q8 = _quantized((tq, hq, d), seed, QD)
     k8 = _quantized((tq, hkv, d), seed + 1, KD)
@@ -45,15 +46,22 @@ def _case(seqlens, hq, hkv, causal, alibi, scale, seed, out_dtype=torch.bfloat16
                                         out_dtype=out_dtype)
     torch.cuda.synchronize()
     assert mea.device_error() == 0
+    return (q8, k8, v8, slopes, cu), out, lse
+
+
+def _check(q8, k8, v8, slopes, seqlens, scale, causal, out, lse):
+    """out [T, Hq, D] / lse [Hq, T] (host or device) of the given e4m3 codes against the oracle
+    of the decoded values, with the bound of the module docstring."""
+    hq, hkv = q8.shape[1], k8.shape[1]
     q = oracle.e4m3_decode(q8.view(torch.uint8)) * QD
     k = oracle.e4m3_decode(k8.view(torch.uint8)) * KD
     v = oracle.e4m3_decode(v8.view(torch.uint8)) * VD
+    c = cu_seqlens(seqlens).tolist()
     sl = None if slopes is None else slopes.double()
-    ref, lref = oracle.attention(q, k, v, cu.tolist(), cu.tolist(), scale, causal, sl)
-    probs = oracle.attention_probs(q, k, v, cu.tolist(), cu.tolist(), scale, causal, sl)
+    ref, lref = oracle.attention(q, k, v, c, c, scale, causal, sl)
+    probs = oracle.attention_probs(q, k, v, c, c, scale, causal, sl)
     r = hq // hkv
     bound = torch.zeros_like(ref)
-    c = cu.tolist()
     for s, pr in enumerate(probs):            # pr [Hq, L, L]
         if pr.numel() == 0:
             continue
@@ -73,6 +81,12 @@ def _case(seqlens, hq, hkv, causal, alibi, scale, seed, out_dtype=torch.bfloat16
     assert torch.equal(torch.isfinite(lg), fin)
     assert float((lg[fin] - lref[fin]).abs().max()) <= 1e-3
     return float(err.max()), float((err / bound).max())
+
+
+def _case(seqlens, hq, hkv, causal, alibi, scale, seed, out_dtype=torch.bfloat16, d=128):
+    (q8, k8, v8, slopes, _), out, lse = _run(seqlens, hq, hkv, causal, alibi, scale, seed,
+                                             out_dtype, d)
+    return _check(q8, k8, v8, slopes, seqlens, scale, causal, out, lse)
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -108,3 +122,25 @@ def test_fp8_rejects_other_head_dims_and_dtypes():
     y = torch.zeros((4, 2, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(mea.MeaError):
         mea.attention_packed_fp8(y, y, y, cu, cu, 4)
+
+
+def test_fp8_packed_workload_full_size_sampled():
+    """The packed prefill workload at full size (32768 tokens in 16 segments, 32/8 heads, D=128,
+    causal + ALiBi) with e4m3 inputs, one launch as the bench runs it; checked whole segment by
+    whole segment (the longest, the shortest and one between) for the four query heads of KV
+    groups 0 and 7, each slice against the oracle with the bound above."""
+    w = workload(2)
+    hq, hkv = 32, 8
+    r = hq // hkv
+    (q8, k8, v8, slopes, cu), out, lse = _run(w.seqlens_q, hq, hkv, True, True, w.scale, w.seed)
+    lens = w.seqlens_q
+    segs = sorted({max(range(len(lens)), key=lambda i: lens[i]),
+                   min(range(len(lens)), key=lambda i: lens[i]), len(lens) // 2})
+    c = cu.tolist()
+    for s in segs:
+        a, e = c[s], c[s + 1]
+        for g in (0, hkv - 1):
+            hs = slice(g * r, (g + 1) * r)
+            _check(q8[a:e, hs], k8[a:e, g:g + 1], v8[a:e, g:g + 1], slopes[hs], [e - a],
+                   w.scale, True, out[a:e, hs], lse[hs, a:e])
+

@@ -121,6 +121,20 @@ def test_workload2_packed_causal_gqa_alibi_full():
     check_packed(w.seqlens_q, w.seqlens_k, 32, 8, 128, w.dtype, True, True, w.scale, w.seed)
 
 
+def test_head_dim_256_long_causal_sampled():
+    # the 16384-token causal prefill at head dim 256 (64/8 heads, scale 1/16), one launch of the
+    # 256-wide kernel at the size the bench times, on sampled rows
+    w = workload(3)
+    (q, k, v, cu_q, cu_k, _), out, lse = run_packed(w.seqlens_q, w.seqlens_k, 64, 8, 256,
+                                                    w.dtype, True, False, 1.0 / 16, w.seed + 256)
+    rows = sample_rows(w.seed + 256, 256, 64, w.total_q, must_tokens=(0, 1, 127, 128, 16383))
+    ro, rl = oracle.attention_rows(q, k, v, cu_q.tolist(), cu_k.tolist(), 1.0 / 16, True, None,
+                                   rows)
+    got = torch.stack([out[t, h].cpu() for h, t in rows])
+    gl = torch.stack([lse[h, t].cpu() for h, t in rows])
+    assert_close(got, ro, gl, rl, w.dtype, "head dim 256, 16384 tokens, sampled rows")
+
+
 def test_workload3_long_causal_sampled():
     w = workload(3)
     (q, k, v, cu_q, cu_k, _), out, lse = run_packed(w.seqlens_q, w.seqlens_k, 64, 8, 128,
