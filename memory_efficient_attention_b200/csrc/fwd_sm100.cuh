@@ -406,34 +406,61 @@ __device__ __forceinline__ bool fwd_softmax_tile(const FwdParams& p, uint32_t t_
     // rarely takes p out of range: exponentiate against it straight away and redo the tile in
     // the rare case it does. The first tile of a row takes its maximum first.
     const bool speculate = __all_sync(0xffffffffu, m_ref != -INFINITY);
-    if (!speculate) {
-      const float m_tile = tile_score_max<ALIBI>(x, p.c1, slope2) + kconst;
-      const float m_new = fmaxf(m_ref, m_tile);
-      resc = m_new > m_ref + 8.0f;
-      if (resc) {
-        alpha = ex2_approx(m_ref - m_new);
-        l *= alpha;
-        m_ref = m_new;
-      }
-    }
-    const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-    float rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_use - kconst, t_s);
-    if (speculate) {
-      // Every p of the tile is at most its row sum, so a sum within the bound keeps every p
-      // within the range P is packed into: 2^15 for 16-bit P (f16 holds up to 65504; bf16 has
-      // fp32's range), 2^8 for e4m3 (448). Otherwise (rare: key tiles are visited from the
-      // diagonal down) take the tile's true maximum and redo the tile against it. The bound
-      // only limits how far the reference maximum may lag; O and l stay in fp32 either way.
-      const bool over = rs > (E8 ? 256.0f : 32768.0f);
-      if (__any_sync(0xffffffffu, over)) {
-        const float m_tile = tile_score_max<ALIBI>(x, p.c1, slope2) + kconst;
-        if (m_tile > m_ref) {
-          resc = true;
-          alpha = ex2_approx(m_ref - m_tile);
-          l *= alpha;
-          m_ref = m_tile;
+    // Every p of the tile is at most its row sum, so a sum within the bound keeps every p within
+    // the range P is packed into: 2^15 for 16-bit P (f16 holds up to 65504; bf16 has fp32's
+    // range), 2^8 for e4m3 (448). Otherwise (rare: key tiles are visited from the diagonal down)
+    // take the tile's true maximum and redo the tile against it. The bound only limits how far
+    // the reference maximum may lag; O and l stay in fp32 either way. (The first tile's maximum
+    // applies the lazy threshold; a redo adopts any larger maximum.)
+    float rs;
+    if constexpr (ALIBI && !E8) {
+      // Both passes in one loop, so that the exponential step (largest with ALiBi) is emitted
+      // once; measured faster with ALiBi and 16-bit P, slower for the other variants, which keep
+      // the two calls below.
+      bool take_max = !speculate;
+      rs = 0.f;
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        if (take_max) {
+          const float m_tile = tile_score_max<ALIBI>(x, p.c1, slope2) + kconst;
+          const float m_new = fmaxf(m_ref, m_tile);
+          if (pass == 0 ? m_new > m_ref + 8.0f : m_tile > m_ref) {
+            resc = true;
+            alpha = ex2_approx(m_ref - m_new);
+            l *= alpha;
+            m_ref = m_new;
+          }
         }
-        rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_ref - kconst, t_s);
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_use - kconst, t_s);
+        if (take_max || !__any_sync(0xffffffffu, rs > 32768.0f)) break;
+        take_max = true;
+      }
+    } else {
+      if (!speculate) {
+        const float m_tile = tile_score_max<ALIBI>(x, p.c1, slope2) + kconst;
+        const float m_new = fmaxf(m_ref, m_tile);
+        resc = m_new > m_ref + 8.0f;
+        if (resc) {
+          alpha = ex2_approx(m_ref - m_new);
+          l *= alpha;
+          m_ref = m_new;
+        }
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_use - kconst, t_s);
+      if (speculate) {
+        const bool over = rs > (E8 ? 256.0f : 32768.0f);
+        if (__any_sync(0xffffffffu, over)) {
+          const float m_tile = tile_score_max<ALIBI>(x, p.c1, slope2) + kconst;
+          if (m_tile > m_ref) {
+            resc = true;
+            alpha = ex2_approx(m_ref - m_tile);
+            l *= alpha;
+            m_ref = m_tile;
+          }
+          rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_ref - kconst, t_s);
+        }
       }
     }
     l += rs;
