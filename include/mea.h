@@ -120,7 +120,8 @@ size_t mea_decode_workspace_size(int n_seqs, int total_k, int n_heads_q, int n_h
  * keys; mask_kind is accepted for symmetry and CAUSAL equals NONE here.
  *   workspace/workspace_bytes: caller-owned device scratch of at least
  *   mea_decode_workspace_size(...) bytes, 256-byte aligned; its contents need no initialisation.
- *   split_keys: keys per chunk, a multiple of 64 (0 = library's choice).
+ *   split_keys: keys per chunk, a multiple of 64 (0 = library's choice: the largest power of
+ *   two from 128 to 2048 that leaves about half a (chunk, head block) work item per SM or more).
  * Two kernels are launched on `stream`: the split kernel and the log-sum-exp merge kernel.
  */
 int mea_decode_splitkv(const void* q, const void* k, const void* v, void* out, float* lse,
