@@ -62,14 +62,17 @@ __device__ __forceinline__ uint32_t dec_row_addr(uint32_t base, int kr, int ch, 
          (static_cast<uint32_t>((ch & 7) ^ (kr & 7)) << 4);
 }
 
-template <int D>
+template <int D, bool PAGED = false>
 struct DecCfg {
   static constexpr int BK = 64;                       // keys per tile
   static constexpr int ATOMS = D / 64;
   static constexpr uint32_t ATOM_BYTES = BK * 128;    // 64 keys x 128 B
   static constexpr uint32_t KT_BYTES = BK * D * 2;    // one K (or V) tile
   static constexpr uint32_t STAGE_BYTES = 2 * KT_BYTES;
-  static constexpr int NS = (D == 256) ? 3 : (D == 128) ? 5 : 8;
+  // Ring stages: at D = 128 the paged cache takes a sixth (its stages arrive as several smaller
+  // boxes, so more of them in flight pay: +2 % on 16-slot blocks), the packed one stays at five
+  // (a sixth measured 0.8 % slower there).
+  static constexpr int NS = (D == 256) ? 3 : (D == 128) ? (PAGED ? 6 : 5) : 8;
   // The four warps' partial O rows are merged through shared memory MC columns at a time.
   static constexpr int MC = D < 128 ? D : 128;
   static constexpr uint32_t SMEM_RING = 0;
@@ -136,7 +139,7 @@ template <int D, bool BF16, bool ALIBI, bool PAGED = false>
 __global__ void __launch_bounds__(160, 1)
     mea_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
-  using C = DecCfg<D>;
+  using C = DecCfg<D, PAGED>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;

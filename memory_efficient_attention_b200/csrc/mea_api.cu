@@ -346,10 +346,10 @@ template <int D, bool BF16, bool ALIBI, bool PAGED>
 int launch_dec_t(const CUtensorMap& tk, const CUtensorMap& tv, const mea::DecParams& p,
                  int grid, int n_kv_heads, cudaStream_t stream) {
   constexpr auto kern = mea::mea_decode_split_kernel<D, BF16, ALIBI, PAGED>;
-  constexpr uint32_t smem = mea::DecCfg<D>::SMEM_TOTAL;
+  constexpr uint32_t smem = mea::DecCfg<D, PAGED>::SMEM_TOTAL;
   if (smem_attr_once<kern>(smem) != cudaSuccess) return MEA_ERR_CUDA;
   clear_stale_launch_error();
-  if (grid > 0) kern<<<grid, mea::DecCfg<D>::THREADS, smem, stream>>>(tk, tv, p);
+  if (grid > 0) kern<<<grid, mea::DecCfg<D, PAGED>::THREADS, smem, stream>>>(tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return MEA_ERR_CUDA;
   dim3 mgrid(p.n_seqs, n_kv_heads);
   mea::mea_lse_merge_kernel<D, BF16><<<mgrid, 256, 0, stream>>>(p);
