@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         tc_fence_after();
         float alpha = 1.f;
-        const bool resc = fwd_softmax_tile<BF16, CAUSAL, ALIBI, false>(
+        const bool resc = fwd_softmax_tile<BF16, CAUSAL, ALIBI, false, true>(
             p, t_lane + b * 128, (n - 1 - jj) * 128, it.lk, pos, p_min, slope2, m_ref, l, alpha);
         if (jj > 0 && __any_sync(0xffffffffu, resc)) {
           // O holds the tiles before this one once the previous P·V has finished.

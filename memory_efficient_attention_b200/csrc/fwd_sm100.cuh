@@ -370,7 +370,7 @@ __device__ __forceinline__ float exp_tile_to_tmem(const float (&x)[128], float c
 // true when O must be rescaled by alpha before this tile's P V.
 //   kv0: key index of column 0; pos: key position of the row; p_min: that of the sub-tile's
 //   first row (rows are ordered by token, so it bounds the diagonal of the whole sub-tile).
-template <bool BF16, bool CAUSAL, bool ALIBI, bool E8>
+template <bool BF16, bool CAUSAL, bool ALIBI, bool E8, bool FOLD = (ALIBI && !E8)>
 __device__ __forceinline__ bool fwd_softmax_tile(const FwdParams& p, uint32_t t_s, int kv0,
                                                  int lk, int pos, int p_min, float slope2,
                                                  float& m_ref, float& l, float& alpha) {
@@ -413,10 +413,10 @@ __device__ __forceinline__ bool fwd_softmax_tile(const FwdParams& p, uint32_t t_
     // the reference maximum may lag; O and l stay in fp32 either way. (The first tile's maximum
     // applies the lazy threshold; a redo adopts any larger maximum.)
     float rs;
-    if constexpr (ALIBI && !E8) {
-      // Both passes in one loop, so that the exponential step (largest with ALiBi) is emitted
-      // once; measured faster with ALiBi and 16-bit P, slower for the other variants, which keep
-      // the two calls below.
+    if constexpr (FOLD) {
+      // Both passes in one loop, so that the exponential step is emitted once; measured faster
+      // with ALiBi and 16-bit P at head dim 128 and in the 256-wide kernel, slower for the other
+      // 128-wide variants, which keep the two calls below.
       bool take_max = !speculate;
       rs = 0.f;
 #pragma unroll 1
@@ -433,7 +433,7 @@ __device__ __forceinline__ bool fwd_softmax_tile(const FwdParams& p, uint32_t t_
         }
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         rs = exp_tile_to_tmem<BF16, ALIBI, E8>(x, p.c1, slope2, m_use - kconst, t_s);
-        if (take_max || !__any_sync(0xffffffffu, rs > 32768.0f)) break;
+        if (take_max || !__any_sync(0xffffffffu, rs > (E8 ? 256.0f : 32768.0f))) break;
         take_max = true;
       }
     } else {
