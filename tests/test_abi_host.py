@@ -127,6 +127,26 @@ def test_decode_workspace_size(lib):
     assert dec(lib, ws=A + 16, split=64) == _lib.MEA_ERR_WORKSPACE
 
 
+@pytest.mark.parametrize("n_seqs,total_k,hq,hkv,chunk", [
+    (64, 1107955, 64, 8, 2048),   # the 64-request decode workload: capped at 2048
+    (8, 83113, 64, 8, 2048),      # its first 8 requests: still 2048
+    (1, 32768, 64, 8, 2048),      # one long request: 128 items for 148 SMs is enough
+    (1, 4096, 64, 8, 256),        # one short request: 2 * 4096 * 8 / 148 = 442 -> 256
+    (1, 512, 64, 8, 128),         # the floor
+    (2, 20000, 16, 16, 2048),     # MHA (one head per item): 16 items per chunk
+])
+def test_decode_automatic_chunk(lib, n_seqs, total_k, hq, hkv, chunk):
+    # With split_keys = 0 the library takes the largest power of two from 128 to 2048 that keeps
+    # about half a (chunk, head block) item per SM or more; head blocks are the largest divisor
+    # of Hq/Hkv up to 16. On a host without a GPU the SM count defaults to 148. The workspace
+    # size identifies the chunk it picked.
+    assert lib.mea_decode_workspace_size(n_seqs, total_k, hq, hkv, 128, 0) == \
+        lib.mea_decode_workspace_size(n_seqs, total_k, hq, hkv, 128, chunk)
+    if chunk < 2048:
+        assert lib.mea_decode_workspace_size(n_seqs, total_k, hq, hkv, 128, 0) != \
+            lib.mea_decode_workspace_size(n_seqs, total_k, hq, hkv, 128, 2 * chunk)
+
+
 def bwd(lib, **kw):
     args = dict(q=A, k=A, v=A, out=A, lse=A, dout=A, dq=A, dk=A, dv=A, cu_q=A, cu_k=A, n_seqs=2,
                 total_q=100, total_k=120, max_q=60, max_k=70, hq=8, hkv=2, d=128, scale=0.1,
