@@ -3,7 +3,8 @@
 // The backward computes dq, dk, dv of L = sum(out * dout) for the forward's definition; its
 // main kernels (tcgen05) are in bwd_tc_sm100.cuh. This file holds the parameter block and
 //   mea_bwd_pre_kernel   per (query head, token) row, one warp per token over its heads
-//                        (HBM-bound: reads out and dout once): nd = -rowsum(dO * O) = -delta and the row's exponent term
+//                        (HBM-bound: reads out and dout once, in whole 128-byte lines at full
+//                        width): nd = -rowsum(dO * O) = -delta and the row's exponent term
 //                        na = -lse log2 e (causal ALiBi: also - slope log2 e ((t - q0) mod 32),
 //                        t - q0 the row's index in its segment), both fp32 in the workspace.
 //                        128 zero rows per head follow the last token, so the tile loops of
@@ -52,6 +53,33 @@ struct BwdParams {
 
 // ------------------------------------------------------------------------------------------
 constexpr int kBwdOrderMax = 1024;
+// pre kernel, full-width rows: heads covered by one 512-byte warp load, and loads of each of
+// out and dout a lane keeps in flight (two: 40 registers, 48 warps per SM; four loads need 64
+// registers and run slower at 32 warps per SM)
+template <int D>
+constexpr int kPreHeadsPerLoad = 256 / D;
+constexpr int kPreBatch = 2;
+
+// sum of the eight products of two 16-byte groups of 16-bit values, in fp32
+template <bool BF16>
+__device__ __forceinline__ float pre_dot8(const uint4 a, const uint4 b) {
+  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+  float acc = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    float2 af, bf;
+    if constexpr (BF16) {
+      af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[u]));
+      bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[u]));
+    } else {
+      af = __half22float2(*reinterpret_cast<const __half2*>(&aw[u]));
+      bf = __half22float2(*reinterpret_cast<const __half2*>(&bw[u]));
+    }
+    acc = fmaf(af.x, bf.x, acc);
+    acc = fmaf(af.y, bf.y, acc);
+  }
+  return acc;
+}
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(128) mea_bwd_pre_kernel(const BwdParams p) {
@@ -97,8 +125,45 @@ __global__ void __launch_bounds__(128) mea_bwd_pre_kernel(const BwdParams p) {
     }
     e_row = __shfl_sync(0xffffffffu, e_row, 0);
   }
-  // Lane h takes head h (and h + 32, ...): the whole row dot product from 16-byte read-only
-  // loads, so that every head's row of the token is in flight at once.
+  const float* lse_t = p.lse + t;
+  if (p.dh == D && p.hq % kPreHeadsPerLoad<D> == 0) {
+    // Full-width rows: a head's row spans D/8 adjacent lanes, so every warp load reads 512
+    // contiguous bytes (whole 128-byte lines, each sector once); the row sums are reduced
+    // over those lanes with shuffles. kPreBatch loads of out and dout are in flight per lane.
+    constexpr int LPH = D / 8;
+    constexpr int HPL = kPreHeadsPerLoad<D>;
+    const size_t row0 = static_cast<size_t>(t) * p.hq * D;
+    const uint4* o4 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.out) + row0) + lane;
+    const uint4* g4 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + row0) + lane;
+    const int n_ld = p.hq / HPL;
+    for (int i0 = 0; i0 < n_ld; i0 += kPreBatch) {
+      uint4 ov[kPreBatch], gv[kPreBatch];
+#pragma unroll
+      for (int b = 0; b < kPreBatch; ++b)
+        if (i0 + b < n_ld) {
+          ov[b] = __ldg(o4 + (i0 + b) * 32);
+          gv[b] = __ldg(g4 + (i0 + b) * 32);
+        }
+#pragma unroll
+      for (int b = 0; b < kPreBatch; ++b) {
+        if (i0 + b >= n_ld) break;
+        float acc = pre_dot8<BF16>(ov[b], gv[b]);
+#pragma unroll
+        for (int o = LPH / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane % LPH == 0) {
+          const int h = (i0 + b) * HPL + lane / LPH;
+          const size_t wi = static_cast<size_t>(h) * p.t_pad + t;
+          float na = -__ldg(lse_t + static_cast<size_t>(h) * p.total_q) * LOG2E;
+          if (p.lin_bias) na = fmaf(-__ldg(p.slopes + h) * LOG2E, static_cast<float>(e_row), na);
+          p.nd[wi] = -acc;
+          p.na[wi] = na;
+        }
+      }
+    }
+    return;
+  }
+  // Other widths: lane h takes head h (and h + 32, ...), the whole row dot product from
+  // 16-byte read-only loads.
   for (int h = lane; h < p.hq; h += 32) {
     const size_t base = (static_cast<size_t>(t) * p.hq + h) * p.dh;
     const uint4* o4 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.out) + base);
@@ -124,7 +189,7 @@ __global__ void __launch_bounds__(128) mea_bwd_pre_kernel(const BwdParams p) {
       }
     }
     const size_t wi = static_cast<size_t>(h) * p.t_pad + t;
-    float na = -__ldg(p.lse + static_cast<size_t>(h) * p.total_q + t) * LOG2E;
+    float na = -__ldg(lse_t + static_cast<size_t>(h) * p.total_q) * LOG2E;
     if (p.lin_bias) na = fmaf(-__ldg(p.slopes + h) * LOG2E, static_cast<float>(e_row), na);
     p.nd[wi] = -acc;
     p.na[wi] = na;
