@@ -132,6 +132,15 @@ def test_backward_dtypes_dims_masks(d, dtype, causal, alibi):
     _check([190, 65], [190, 65], 4, 2, d, dtype, causal, alibi, 0.11, 950)
 
 
+@pytest.mark.parametrize("hq,hkv,d", [(6, 2, 64), (12, 4, 64), (1, 1, 128), (2, 1, 128),
+                                      (3, 1, 128)])
+def test_backward_row_term_paths(hq, hkv, d):
+    # full-width rows are read as 512-byte warp loads when the heads fill them (a multiple of
+    # 256 / D heads), else one lane per head: both forms, at both kernel widths
+    _check([190, 65, 3], [190, 65, 3], hq, hkv, d, torch.bfloat16, True, True,
+           1 / math.sqrt(d), 990 + hq + d)
+
+
 @pytest.mark.parametrize("d", [8, 32, 40, 72, 96, 120])
 def test_backward_other_head_dims(d):
     # multiples of 8 up to 128: the 64- or 128-wide kernels with zero-filled columns
