@@ -487,6 +487,11 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       using OutT = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const bool any = n_iter > 0;
       const size_t o = (static_cast<size_t>(k0 + key) * p.hkv + g) * p.dh;
+      // 32-byte stores (whole sectors, half the store instructions of 16-byte ones) while the
+      // rows stay 32-byte aligned
+      const bool kv_al32 =
+          ((reinterpret_cast<uintptr_t>(p.dk) | reinterpret_cast<uintptr_t>(p.dv)) & 31) == 0 &&
+          (p.dh & 15) == 0;
       // the first half of the groups writes dV, the second half scale * dK, each group its
       // share of the D columns
       constexpr int HALF = C::NWG / 2 > 0 ? C::NWG / 2 : 1;
@@ -508,11 +513,17 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
             pa[u] = any ? bpack2<BF16>(__uint_as_float(a[2 * u]) * mul,
                                        __uint_as_float(a[2 * u + 1]) * mul)
                         : 0u;
-          uint4* dp4 = reinterpret_cast<uint4*>(dst + c * 32);
+          if (kv_al32) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (c * 32 + u * 8 < p.dh)
-              dp4[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
+            for (int i = 0; i < 2; ++i)
+              if (c * 32 + i * 16 < p.dh) st_global_v8(dst + c * 32 + i * 16, &pa[8 * i]);
+          } else {
+            uint4* dp4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (c * 32 + u * 8 < p.dh)
+                dp4[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
+          }
         }
       }
     }
@@ -824,6 +835,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const bool any = n_jt > 0;
+      // 32-byte stores while the rows stay 32-byte aligned (as for dK/dV)
+      const bool dq_al32 = (reinterpret_cast<uintptr_t>(p.dq) & 31) == 0 && (p.dh & 15) == 0;
       if (wg < D / 32) {
         uint32_t a[32];
         tmem_ld32(t_lane + T_DQ + wg * 32, a);
@@ -836,11 +849,18 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::THREADS, 1)
                                        __uint_as_float(a[2 * u + 1]) * p.scale)
                         : 0u;
           const size_t o = (static_cast<size_t>(q0 + row) * p.hq + h) * p.dh;
-          uint4* dqp = reinterpret_cast<uint4*>(reinterpret_cast<OutT*>(p.dq) + o + wg * 32);
+          OutT* dqrow = reinterpret_cast<OutT*>(p.dq) + o + wg * 32;
+          if (dq_al32) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (wg * 32 + u * 8 < p.dh)
-              dqp[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
+            for (int i = 0; i < 2; ++i)
+              if (wg * 32 + i * 16 < p.dh) st_global_v8(dqrow + i * 16, &pa[8 * i]);
+          } else {
+            uint4* dqp = reinterpret_cast<uint4*>(dqrow);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (wg * 32 + u * 8 < p.dh)
+                dqp[u] = make_uint4(pa[4 * u], pa[4 * u + 1], pa[4 * u + 2], pa[4 * u + 3]);
+          }
         }
       }
       // dQ has been read out of TMEM: the next item may accumulate over it

@@ -141,6 +141,40 @@ def test_backward_row_term_paths(hq, hkv, d):
            1 / math.sqrt(d), 990 + hq + d)
 
 
+def test_backward_outputs_16_byte_aligned_only():
+    """dq, dk, dv whose base addresses are 16 but not 32 bytes aligned take the 16-byte store
+    form of the epilogues: the same values, bit for bit, as 32-byte aligned outputs, and within
+    the derived bound of the oracle."""
+    lens, hq, hkv, d, scale = [190, 65, 3], 8, 2, 128, 1 / math.sqrt(128)
+    (q, k, v, dout, cq, ck, slopes), ref_al = _run(lens, lens, hq, hkv, d, torch.bfloat16, True,
+                                                   True, scale, 996)
+    dev = "cuda"
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, dout))
+    cqd, ckd, sd = cq.to(dev), ck.to(dev), slopes.to(dev)
+    out, lse = mea.attention_packed(qd, kd, vd, cqd, ckd, max(lens), causal=True,
+                                    alibi_slopes=sd, scale=scale)
+
+    def offset_empty(shape):
+        n = math.prod(shape)
+        buf = torch.empty(n + 8, dtype=torch.bfloat16, device=dev)  # 8 elements = 16 bytes
+        t = buf[8:].view(shape)
+        assert t.data_ptr() % 32 == 16
+        return t
+
+    dq, dk, dv = offset_empty(qd.shape), offset_empty(kd.shape), offset_empty(vd.shape)
+    mea.attention_packed_backward(qd, kd, vd, out, lse, dod, cqd, ckd, max(lens), max(lens),
+                                  causal=True, alibi_slopes=sd, scale=scale, dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert mea.device_error() == 0
+    got = (dq.cpu(), dk.cpu(), dv.cpu())
+    for g, r in zip(got, ref_al):
+        assert torch.equal(g, r)
+    sl = slopes.double()
+    ref = oracle.attention_backward(q, k, v, dout, cq.tolist(), ck.tolist(), scale, True, sl)
+    bounds = grad_bounds(q, k, v, dout, cq.tolist(), ck.tolist(), scale, True, sl, torch.bfloat16)
+    _assert_grad_close(got, ref, bounds, "16-byte aligned outputs")
+
+
 @pytest.mark.parametrize("d", [8, 32, 40, 72, 96, 120])
 def test_backward_other_head_dims(d):
     # multiples of 8 up to 128: the 64- or 128-wide kernels with zero-filled columns
